@@ -1,0 +1,478 @@
+#!/usr/bin/env python
+"""Benchmark: GPTQ+QEP layers quantised per second on one Llama-2-7B-shaped layer.
+
+One step = the whole per-layer path on one synthetic layer already resident in
+HBM: H = 2 Xhat^T Xhat (oc_hessian_accumulate), the QEP correction
+(oc_qep_correct with that H) and GPTQ with packing (oc_gptq_quantize).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Under torchrun every rank quantises its own
+layer (independent problems, no collective on the data path): weak scaling,
+value = layers of all ranks / max-over-ranks device time.  ``--impl reference``
+times the float64 CPU oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GPTQ+QEP layers quantized/sec (Llama-7B shapes, 4-bit g128); % of roofline"
+UNIT = "layers/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+SM_COUNT = 148
+CPU_SAMPLE_TOKENS = 4096
+CPU_SAMPLE_ROWS = 1024
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(spec):
+    return {
+        "workload": (f"{spec.name}: Llama-2-7B q_proj layer {spec.d_out}x{spec.d_in}, "
+                     f"{spec.n_tok} calibration tokens (bf16 Student-t(4), 1% channels x20, "
+                     f"Xhat = X + 2% channel noise), QEP alpha {spec.alpha}, GPTQ "
+                     f"{spec.wbits}-bit g{spec.groupsize} asymmetric, damp {spec.damp}, "
+                     f"act_order {'on' if spec.act_order else 'off'}"),
+        "d_out": spec.d_out, "d_in": spec.d_in, "n_tok": spec.n_tok, "wbits": spec.wbits,
+        "groupsize": spec.groupsize, "act_order": spec.act_order,
+        "l2": "inputs larger than L2 (X and Xhat are 2.1 GB each), no flush needed",
+    }
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, smax, reasons = [], [], set()
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_index_for(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+
+def phase_work(spec):
+    """Algorithmic work of each phase of one layer: (amount, unit, bound)."""
+    n, m, N = spec.d_in, spec.d_out, spec.n_tok
+    G = spec.d_in if spec.groupsize == -1 else spec.groupsize
+    trailing = sum(2 * m * min(128, n - j1) * (n - j1 - min(128, n - j1)) for j1 in range(0, n, 128))
+    return {
+        # symmetric half of X^T X: n(n+1)/2 entries x 2N flops
+        "hessian_syrk": (n * (n + 1) * N, "flop", "tensor"),
+        "qep_cross": (2 * n * n * N, "flop", "tensor"),
+        "qep_w_delta": (2 * m * n * n, "flop", "f32"),
+        # one Cholesky (n^3/3) + one triangular inverse (n^3/3), for QEP and again for GPTQ
+        "factor": (2 * (2 * n ** 3 // 3), "flop", "f32"),
+        "qep_apply": (2 * m * n * n, "flop", "f32"),
+        "gptq_trailing": (trailing, "flop", "f32"),
+        # read W (fp32) once, write codes (u8) and block errors (fp32)
+        "gptq_sweep": (m * n * 4 + m * n + m * n * 4, "byte", "hbm"),
+        "gptq_prep": (2 * m * n * 4, "byte", "hbm"),
+        "gptq_pack": (m * n + m * n * spec.wbits // 8 + m * (n // G) * 8, "byte", "hbm"),
+    }
+
+
+def f32_simt_peak_tflops(sm_mhz):
+    # 148 SMs x 128 fp32 lanes x 2 flop per FMA x clock
+    return SM_COUNT * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def time_oracle_layer(spec, n_sample=CPU_SAMPLE_TOKENS, m_sample=CPU_SAMPLE_ROWS):
+    """Time the float64 oracle on a bounded sample of one layer.
+
+    The oracle's public pieces are timed separately and each is scaled by the
+    part of the workload it is proportional to: the Hessian and the QEP cross
+    product run on ``n_sample`` tokens (scaled to the workload's tokens); the
+    QEP solve/apply and the GPTQ sweep run on ``m_sample`` rows of W (scaled
+    to d_out); the factorisations run in full.  Returns (seconds per layer,
+    seconds actually measured).
+    """
+    import numpy as np
+
+    import oracle
+    from synthetic import make_layer_host
+
+    L = make_layer_host(spec, n_tok=n_sample)
+    W = L["W"].astype(np.float64)
+    Ws = W[:m_sample]
+    tok_scale = spec.n_tok / n_sample
+    row_scale = spec.d_out / m_sample
+    clock = time.perf_counter
+    t0 = clock()
+    H = oracle.hessian(L["Xhat"])
+    t_h = clock() - t0
+    t0 = clock()
+    oracle.qep_cross(L["X"], L["Xhat"])
+    t_x = clock() - t0
+    t0 = clock()
+    oracle.qep_correct(W[:0], L["X"], L["Xhat"], spec.alpha, spec.damp, H=H)
+    t_q0 = clock() - t0  # cross product + factorisation, no rows
+    t0 = clock()
+    Wps = oracle.qep_correct(Ws, L["X"], L["Xhat"], spec.alpha, spec.damp, H=H)
+    t_qm = clock() - t0
+    t0 = clock()
+    prep = oracle.gptq_prepare(Wps, H, spec.damp, spec.act_order)
+    U = oracle.inv_chol_upper(prep["Hd"])
+    t_f = clock() - t0
+    t0 = clock()
+    oracle.gptq_sweep(prep["W"], U, spec.wbits, spec.groupsize, prep["perm"])
+    t_s = clock() - t0
+    total = ((t_h + t_x) * tok_scale + (t_q0 - t_x) + max(0.0, t_qm - t_q0) * row_scale
+             + t_f + t_s * row_scale)
+    measured = t_h + t_x + t_q0 + t_qm + t_f + t_s
+    return total, measured
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        th = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if th:
+            return max(th)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_sample_text(spec, n_sample=CPU_SAMPLE_TOKENS, m_sample=CPU_SAMPLE_ROWS):
+    return (f"{n_sample} of {spec.n_tok} calibration tokens for the Hessian and QEP cross product "
+            f"(scaled x{spec.n_tok / n_sample:g}); {m_sample} of {spec.d_out} rows for the QEP "
+            f"apply and the GPTQ sweep (scaled x{spec.d_out / m_sample:g}); both factorisations of "
+            f"the {spec.d_in}x{spec.d_in} Hessian in full; inputs from the host recipe of the workload")
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import post_weight_quantization_07_b200 as oc
+    from synthetic import CONFIGS, make_layer_device
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    spec = CONFIGS[args.workload]
+    if args.n_tok:
+        spec = spec.with_(n_tok=args.n_tok)
+    spec_r = spec.with_(seed=spec.seed + 1000 * rank)
+    L = make_layer_device(spec_r, "cuda")
+    W, X, Xh = L["W"], L["X"], L["Xhat"]
+    m, n = spec.d_out, spec.d_in
+    G = n if spec.groupsize == -1 else spec.groupsize
+    H = torch.zeros(n, n, device="cuda")
+    Wp = torch.empty_like(W)
+    codes = torch.empty(m, n * spec.wbits // 32, dtype=torch.int32, device="cuda")
+    scales = torch.empty(m, n // G, device="cuda")
+    zeros = torch.empty(m, n // G, device="cuda")
+    stream = torch.cuda.current_stream()
+    oc.oc_set_sync(False)
+
+    def step():
+        H.zero_()
+        oc.oc_hessian_accumulate(Xh, H, stream=stream)
+        oc.oc_qep_correct(W, X, Xh, spec.alpha, spec.damp, H_opt=H, W_out=Wp, stream=stream)
+        oc.oc_gptq_quantize(Wp, H, spec.wbits, spec.groupsize, spec.damp, spec.act_order,
+                            codes=codes, scales=scales, zeros=zeros, stream=stream)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    st = oc.oc_stream_status(stream)
+    if st != oc.OC_OK:
+        raise RuntimeError(f"warm-up failed: {oc.oc_status_string(st)}")
+
+    # ---- device-timed region: inputs resident in HBM
+    oc.oc_profile_read()
+    oc.oc_profile_enable(True)
+    launches0 = oc.oc_launch_count()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_index_for(local_rank)) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        barrier()
+    launches = oc.oc_launch_count() - launches0
+    oc.oc_profile_enable(False)
+    phases = oc.oc_profile_read()
+    st = oc.oc_stream_status(stream)
+    if st != oc.OC_OK:
+        raise RuntimeError(f"timed steps failed: {oc.oc_status_string(st)}")
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_per_step = ms_total / args.steps
+    value = world * args.steps / (ms_total / 1e3)
+
+    # ---- end to end: pinned host inputs copied in and results read back every step
+    e2e = None
+    if not args.no_e2e:
+        Xh_h = torch.empty(Xh.shape, dtype=Xh.dtype, pin_memory=True)
+        X_h = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
+        W_h = torch.empty(W.shape, dtype=W.dtype, pin_memory=True)
+        Xh_h.copy_(Xh)
+        X_h.copy_(X)
+        W_h.copy_(W)
+        codes_h = torch.empty(codes.shape, dtype=codes.dtype, pin_memory=True)
+        scales_h = torch.empty(scales.shape, dtype=scales.dtype, pin_memory=True)
+        zeros_h = torch.empty(zeros.shape, dtype=zeros.dtype, pin_memory=True)
+
+        def e2e_step():
+            Xh.copy_(Xh_h, non_blocking=True)
+            X.copy_(X_h, non_blocking=True)
+            W.copy_(W_h, non_blocking=True)
+            step()
+            codes_h.copy_(codes, non_blocking=True)
+            scales_h.copy_(scales, non_blocking=True)
+            zeros_h.copy_(zeros, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        k2 = max(1, min(args.steps, 5))
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(k2):
+            e2e_step()
+        f1.record(stream)
+        barrier()
+        st = oc.oc_stream_status(stream)
+        if st != oc.OC_OK:
+            raise RuntimeError(f"end-to-end steps failed: {oc.oc_status_string(st)}")
+        ms_e2e = max_over_ranks(f0.elapsed_time(f1))
+        h2d = Xh.numel() * Xh.element_size() + X.numel() * X.element_size() + W.numel() * 4
+        d2h = codes.numel() * 4 + scales.numel() * 4 + zeros.numel() * 4
+        e2e = {"value": world * k2 / (ms_e2e / 1e3), "unit": UNIT, "steps": k2,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    clocks = clk.summary()
+    work = phase_work(spec)
+    phase_out = {}
+    for name, (ms, nl) in phases.items():
+        if nl == 0 and ms == 0.0:
+            continue
+        amt, unit, bound = work.get(name, (0, "", ""))
+        ms_step = ms / args.steps
+        entry = {"ms_per_step": round(ms_step, 4), "launches_per_step": nl / args.steps}
+        if amt and ms_step > 0:
+            if unit == "flop":
+                entry["achieved_tflops"] = round(amt / (ms_step / 1e3) / 1e12, 2)
+            else:
+                entry["achieved_gbs"] = round(amt / (ms_step / 1e3) / 1e9, 1)
+            entry["bound"] = bound
+        phase_out[name] = entry
+
+    # dominant kernel = the phase with the largest device time
+    dom = max(phase_out, key=lambda k: phase_out[k]["ms_per_step"])
+    amt, unit, bound = work[dom]
+    launches_dom = max(1.0, phase_out[dom]["launches_per_step"])
+    ms_launch = phase_out[dom]["ms_per_step"] / launches_dom
+    per_launch = amt / launches_dom
+    sm_mhz = clocks.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+    if bound == "tensor":
+        peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        achieved = per_launch / (ms_launch / 1e3) / 1e12
+        roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_source": f"{peak_src} bf16 sustained"}
+    elif bound == "f32":
+        peak = f32_simt_peak_tflops(sm_mhz)
+        achieved = per_launch / (ms_launch / 1e3) / 1e12
+        roof = {"bound": "alu", "unit": "TFLOP/s",
+                "peak_source": f"fp32 CUDA-core FMA peak at the sampled {sm_mhz:.0f} MHz (148 SM x 128 lanes x 2)"}
+    else:
+        peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        achieved = per_launch / (ms_launch / 1e3) / 1e9
+        roof = {"bound": "hbm", "unit": "GB/s", "peak_source": f"{peak_src} HBM copy"}
+    roof.update({"kernel_phase": dom, "achieved": round(achieved, 2), "peak": round(peak, 2),
+                 "frac": round(achieved / peak, 4), "traffic": None,
+                 "per_launch": {"amount": per_launch, "unit": unit, "ms": round(ms_launch, 4)}})
+
+    # whole-layer roofline time: tensor phases at the bf16 peak, f32 phases at the
+    # fp32 peak of the tensor cores' 3xTF32 path is not used here: each phase at
+    # the peak of the unit it runs on today
+    t_roof = 0.0
+    for name, (amt, unit, bound) in work.items():
+        if bound == "tensor":
+            t_roof += amt / (peaks.get("bf16_tflops_sustained", 1400.0) * 1e12)
+        elif bound == "f32":
+            t_roof += amt / (f32_simt_peak_tflops(sm_mhz) * 1e12)
+        else:
+            t_roof += amt / (peaks.get("hbm_gbs", 6650.0) * 1e9)
+
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16+f32",
+        "data": "synthetic",
+        "config": dict(workload_config(spec),
+                       parallelism=(f"{world} independent layers, one per rank" if world > 1
+                                    else "single GPU")),
+        "seconds_per_224_layers_of_this_shape": round(224 * ms_per_step / 1e3, 3),
+        "layer_roofline_ms_current_units": round(t_roof * 1e3, 3),
+        "roofline": roof, "phases": phase_out, "gpu_launches": int(launches),
+        "clocks": clocks, "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        t_layer, t_meas = time_oracle_layer(spec)
+        line["cpu_baseline"] = {"value": round(1.0 / t_layer, 6), "unit": UNIT,
+                                "cores": blas_threads(), "kind": "oracle",
+                                "sample": cpu_sample_text(spec),
+                                "cpu_seconds_measured": round(t_meas, 2)}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from synthetic import CONFIGS
+    spec = CONFIGS[args.workload]
+    if args.n_tok:
+        spec = spec.with_(n_tok=args.n_tok)
+    for _ in range(args.warmup):
+        time_oracle_layer(spec, n_sample=512, m_sample=64)
+    times = []
+    measured = 0.0
+    for _ in range(args.steps):
+        t, tm = time_oracle_layer(spec)
+        times.append(t)
+        measured += tm
+    t = statistics.median(times)
+    value = 1.0 / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(workload_config(spec), parallelism="host cores"),
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": blas_threads(),
+                         "kind": "oracle", "sample": cpu_sample_text(spec),
+                         "cpu_seconds_measured": round(measured, 2)},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c2_q_proj")
+    ap.add_argument("--n-tok", type=int, default=None,
+                    help="calibration tokens per layer (default: the workload's own)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

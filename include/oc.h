@@ -1,0 +1,187 @@
+/*
+ * oc.h -- C ABI of liboc.so: layer-wise GPTQ + QEP weight quantisation on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the quantisation pipeline of the OneComp pages:
+ *   - the OneComp v1.1.0 release summary (easyvibecoding.app/curated/1062),
+ *     section "量化錯誤傳播 (QEP)": Quantization Error Propagation corrects a
+ *     layer's weights for the quantisation error of the layers before it;
+ *     section "v1.1.0全新量化方法": group quantisation, e.g. 4-bit, groupsize 128;
+ *   - the One Compression hub page (pomoai.com/hubs/FujitsuResearch/OneCompression),
+ *     section "核心功能拆解", quantiser table: GPTQ, 2-4 bit Hessian-optimal
+ *     rounding; API GPTQ(wbits, groupsize) with qep=True.
+ * The pages print no equations; each call below states what it computes.
+ *
+ * Conventions shared by every call
+ *   - All array arguments are DEVICE pointers on the current CUDA device,
+ *     owned by the caller, row-major, densely packed (leading dimension = the
+ *     number of columns).  The library never frees or retains them.
+ *   - Calibration activations are token-major bf16 (the PyTorch activation
+ *     layout): X[t * n + c] is channel c of token t.
+ *   - W is d_out x d_in = m x n fp32.  n must be a positive multiple of 64
+ *     (at most 49152 for QEP and GPTQ); m >= 1.  Pointers handed to the
+ *     tensor-memory-access (TMA) paths (X, Xhat, H, W, codes) must be 16-byte aligned.
+ *   - The stream argument is a cudaStream_t (NULL = legacy default stream).
+ *     All work of a call is ordered on that stream.
+ *   - The library owns one scratch workspace per device, grown on demand with
+ *     cudaMalloc (which synchronises the device when it grows) and released by
+ *     oc_workspace_release().  Calls that share a device must not overlap in
+ *     time (they share the workspace and the device status word).
+ *   - Return value: an oc_status.  Argument errors are detected on the host
+ *     before anything is launched.  Errors found on the device (a non-positive
+ *     pivot, a non-finite value, a bounded wait that ran out) are recorded in a
+ *     device status word; in synchronous mode (the default) each call
+ *     synchronises its stream and returns that status.  In asynchronous mode
+ *     (oc_set_sync(0)) calls return OC_OK after launching and
+ *     oc_stream_status() synchronises and reports the first recorded error.
+ *   - oc_last_error() gives a human-readable detail of the last failure on the
+ *     calling thread.
+ */
+#ifndef OC_H
+#define OC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  OC_OK = 0,
+  OC_ERR_INVALID_ARG = 1,  /* null pointer, bad size, unsupported combination of arguments */
+  OC_ERR_UNSUPPORTED = 2,  /* valid request this build does not handle (e.g. not sm_100) */
+  OC_ERR_NOT_SPD = 3,      /* a Cholesky pivot was <= 0: the (dampened) Hessian is not SPD */
+  OC_ERR_NONFINITE = 4,    /* a NaN or Inf was met in an input or an intermediate */
+  OC_ERR_TIMEOUT = 5,      /* a bounded on-device wait ran out (kernel gave up cleanly) */
+  OC_ERR_CUDA = 6,         /* a CUDA runtime call failed; see oc_last_error() */
+  OC_ERR_OOM = 7           /* the workspace could not be grown */
+} oc_status;
+
+/* Name of a status code ("OC_OK", ...). Never NULL. */
+const char* oc_status_string(int status);
+
+/* Detail text of the last failure on the calling thread ("" if none). */
+const char* oc_last_error(void);
+
+/* ABI version of this library (major * 100 + minor). */
+int oc_version(void);
+
+/* 1 (default): every call synchronises its stream and returns the device status.
+ * 0: calls return after launching; use oc_stream_status() to collect errors. */
+void oc_set_sync(int sync);
+
+/* Synchronise `stream`, return the first device-side error recorded since the
+ * last collection, and clear it. */
+int oc_stream_status(void* stream);
+
+/* Free this device's workspace (synchronises the device). */
+int oc_workspace_release(void);
+
+/* Per-phase device timing, for benchmarking.  When enabled, every phase of a
+ * call (see oc_profile_phase_name) records a pair of CUDA events on the call's
+ * stream around its kernels.  Off by default. */
+int oc_profile_enable(int on);
+
+/* Wait for the recorded events and write, per phase, the milliseconds and the
+ * kernel launches accumulated since the last read into ms[0..max_phases) and
+ * launches[0..max_phases) (either may be NULL); clears the record.  Returns
+ * the number of phases. */
+int oc_profile_read(double* ms, int64_t* launches, int max_phases);
+
+/* Name of phase `phase` ("" when out of range). */
+const char* oc_profile_phase_name(int phase);
+
+/* Kernel launches made by this library since it was loaded. */
+int64_t oc_launch_count(void);
+
+/*
+ * Hessian accumulation:  H += 2 * X^T X   (n x n, fp32)
+ *
+ * The Hessian of the layer-wise loss ||(W - Q) X^T||_F^2 with respect to a
+ * row of the weights -- the matrix behind GPTQ's "Hessian-optimal rounding"
+ * (One Compression hub page, section "核心功能拆解", quantiser table, GPTQ row).
+ * Pass the inputs the quantised layer will see (X-hat); repeated calls over
+ * token chunks accumulate (chunked calibration).
+ *
+ *   X      bf16 [n_tok x n], token-major (device).  Read only.
+ *   n_tok  number of tokens, 0 <= n_tok < 2^31 - 64 (0 leaves H unchanged and X may be NULL).
+ *   n      number of input channels (d_in), positive multiple of 64.
+ *   H      fp32 [n x n] (device), read-modify-write.  Must be symmetric on entry
+ *          (e.g. zeros, or the output of a previous call): the update is
+ *          computed for the upper triangle, added in place, and the lower
+ *          triangle is then overwritten with the mirror of the upper one.
+ * Products are exact (bf16 x bf16 in fp32) and accumulated in fp32 on the
+ * tensor cores (tcgen05, TMEM accumulators), split over token chunks whose
+ * partial sums are added into H in fp32 (summation order not fixed).
+ */
+int oc_hessian_accumulate(const void* X, int64_t n_tok, int64_t n, float* H, void* stream);
+
+/*
+ * QEP weight correction (OneComp release summary, section "量化錯誤傳播 (QEP)"):
+ *
+ *   W_out = W + alpha * W d A^-1,   d = (X - Xhat)^T Xhat,
+ *   A = Xhat^T Xhat + lam I,        lam = damp * mean(diag(Xhat^T Xhat)).
+ *
+ * W + W d A^-1 is the minimiser of ||W X^T - W' Xhat^T||_F^2 + lam ||W' - W||_F^2:
+ * the weight that, fed the perturbed inputs Xhat, best reproduces the
+ * full-precision output; alpha in [0, 1] moves that fraction of the way.
+ * alpha == 0 returns W unchanged, bit for bit.
+ *
+ *   W      fp32 [m x n] (device), read only.
+ *   X      bf16 [n_tok x n] full-precision inputs (device).
+ *   Xhat   bf16 [n_tok x n] inputs the quantised layer sees (device).
+ *   n_tok  >= 1.
+ *   alpha  finite.   damp  >= 0 (damp == 0 requires Xhat^T Xhat to be SPD).
+ *   H_opt  NULL, or fp32 [n x n] = 2 Xhat^T Xhat over the same tokens (from
+ *          oc_hessian_accumulate); it then replaces the recomputation.
+ *   W_out  fp32 [m x n] (device); may equal W (in place).
+ * Errors: OC_ERR_NOT_SPD if A is not positive definite.
+ */
+int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const void* Xhat,
+                   int64_t n_tok, float alpha, float damp, const float* H_opt,
+                   float* W_out, void* stream);
+
+/*
+ * GPTQ quantisation with a per-group asymmetric min/max grid (One Compression
+ * hub page, section "核心功能拆解": GPTQ 2-4 bit Hessian-optimal rounding,
+ * GPTQ(wbits, groupsize); OneComp release summary, section "v1.1.0全新量化方法":
+ * 4-bit, groupsize 128).  Steps:
+ *   1. dead columns (H_jj == 0): H_jj := 1 and W[:, j] := 0;
+ *   2. act_order: process columns by a stable descending sort of diag(H);
+ *   3. H_d = H + damp * mean(diag H) * I;  U = upper Cholesky factor of H_d^-1;
+ *   4. sweep columns in processing order: q = clip(rint(w/scale) + zero, 0, 2^b-1),
+ *      e = (w - scale (q - zero)) / U_jj, later columns w_k -= e U_jk
+ *      (inside blocks of 128 columns; a tensor-core GEMM applies each block's
+ *      errors to all later columns);
+ *   5. grid: scale = (max - min) / (2^b - 1), zero = clip(rint(-min/scale), 0, 2^b-1)
+ *      over the group's values (min = max widens to [min-1, max+1]); without
+ *      act_order taken at the group's first column from its current values,
+ *      with act_order taken up front from W (after step 1); groups are
+ *      contiguous in original column order;
+ *   6. codes are packed per row as an LSB-first bitstream of wbits-bit codes
+ *      along d_in in original column order (wbits = 3 crosses word boundaries).
+ *
+ *   W          fp32 [m x n] (device), read only (the library works on a copy).
+ *   H          fp32 [n x n] symmetric (device), read only.
+ *   wbits      2, 3 or 4.
+ *   groupsize  -1 (one group per row), or a power of two 4..128 dividing n, or a
+ *              multiple of 128 dividing n.
+ *   damp       >= 0.   act_order  0 or 1.
+ *   codes      uint32 [m x (n * wbits / 32)] (device), written.
+ *   scales     fp32 [m x n/G] (device), written.   zeros  fp32 [m x n/G], integer
+ *              valued, written.  (G = n when groupsize == -1.)
+ *   perm_out   NULL, or int32 [n] (device): the processing order as original
+ *              column indices (identity without act_order).
+ * Errors: OC_ERR_NOT_SPD if H_d is not positive definite, OC_ERR_NONFINITE for
+ * non-finite entries of diag(H).
+ */
+int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int wbits,
+                     int groupsize, float damp, int act_order, uint32_t* codes,
+                     float* scales, float* zeros, int32_t* perm_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OC_H */

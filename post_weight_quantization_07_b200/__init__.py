@@ -1,0 +1,230 @@
+"""B200-native layer-wise GPTQ + QEP weight quantisation.
+
+Python binding of ``liboc.so`` (the C ABI in ``include/oc.h``).  The functions
+below carry the C names and only marshal arguments: they check dtypes,
+shapes and devices of torch tensors, allocate outputs the caller did not
+supply, and pass raw device pointers and the current CUDA stream to the
+library, whose kernels do every step of the computation.  The library is
+loaded on first use; if it has not been built that first use raises an
+ImportError with an explanation (there is no fallback implementation).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+__all__ = ["OC_OK", "OC_ERR_INVALID_ARG", "OC_ERR_UNSUPPORTED", "OC_ERR_NOT_SPD",
+           "OC_ERR_NONFINITE", "OC_ERR_TIMEOUT", "OC_ERR_CUDA", "OC_ERR_OOM", "OcError",
+           "LIB_PATH", "HEADER_PATH", "lib", "declared_symbols", "oc_hessian_accumulate",
+           "oc_qep_correct", "oc_gptq_quantize", "oc_set_sync", "oc_stream_status",
+           "oc_workspace_release", "oc_status_string", "oc_last_error", "oc_version",
+           "oc_profile_enable", "oc_profile_read", "oc_launch_count"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liboc.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "oc.h")
+
+OC_OK = 0
+OC_ERR_INVALID_ARG = 1
+OC_ERR_UNSUPPORTED = 2
+OC_ERR_NOT_SPD = 3
+OC_ERR_NONFINITE = 4
+OC_ERR_TIMEOUT = 5
+OC_ERR_CUDA = 6
+OC_ERR_OOM = 7
+
+
+class OcError(RuntimeError):
+    """A liboc call returned a status other than OC_OK."""
+
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {_status_name(status)} ({detail})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m post_weight_quantization_07_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, f32, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
+    L.oc_status_string.argtypes = [i32]
+    L.oc_status_string.restype = ctypes.c_char_p
+    L.oc_last_error.argtypes = []
+    L.oc_last_error.restype = ctypes.c_char_p
+    L.oc_version.argtypes = []
+    L.oc_version.restype = i32
+    L.oc_set_sync.argtypes = [i32]
+    L.oc_set_sync.restype = None
+    L.oc_stream_status.argtypes = [vp]
+    L.oc_stream_status.restype = i32
+    L.oc_workspace_release.argtypes = []
+    L.oc_workspace_release.restype = i32
+    L.oc_profile_enable.argtypes = [i32]
+    L.oc_profile_enable.restype = i32
+    L.oc_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64), i32]
+    L.oc_profile_read.restype = i32
+    L.oc_profile_phase_name.argtypes = [i32]
+    L.oc_profile_phase_name.restype = ctypes.c_char_p
+    L.oc_launch_count.argtypes = []
+    L.oc_launch_count.restype = i64
+    L.oc_hessian_accumulate.argtypes = [vp, i64, i64, vp, vp]
+    L.oc_hessian_accumulate.restype = i32
+    L.oc_qep_correct.argtypes = [vp, i64, i64, vp, vp, i64, f32, f32, vp, vp, vp]
+    L.oc_qep_correct.restype = i32
+    L.oc_gptq_quantize.argtypes = [vp, i64, i64, vp, i32, i32, f32, i32, vp, vp, vp, vp, vp]
+    L.oc_gptq_quantize.restype = i32
+    return L
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        _LIB = _load()
+    return _LIB
+
+
+def __getattr__(name):
+    # ``post_weight_quantization_07_b200.lib`` is the loaded ctypes library
+    if name == "lib":
+        return _lib()
+    raise AttributeError(name)
+
+
+def declared_symbols():
+    """Names of the functions ``include/oc.h`` declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+(oc_\w+)\s*\(", text, re.M)))
+
+
+def _status_name(status: int) -> str:
+    return _lib().oc_status_string(int(status)).decode()
+
+
+def oc_status_string(status: int) -> str:
+    return _status_name(status)
+
+
+def oc_last_error() -> str:
+    return _lib().oc_last_error().decode()
+
+
+def oc_version() -> int:
+    return _lib().oc_version()
+
+
+def oc_set_sync(sync: bool) -> None:
+    _lib().oc_set_sync(1 if sync else 0)
+
+
+def _check(status: int, where: str):
+    if status != OC_OK:
+        raise OcError(status, where, oc_last_error())
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def oc_stream_status(stream=None) -> int:
+    return _lib().oc_stream_status(_stream_handle(stream))
+
+
+def oc_profile_enable(on: bool) -> None:
+    _check(_lib().oc_profile_enable(1 if on else 0), "oc_profile_enable")
+
+
+def oc_profile_read():
+    """{phase name: (milliseconds, kernel launches)} accumulated since the last read."""
+    k = 32
+    ms = (ctypes.c_double * k)()
+    ln = (ctypes.c_int64 * k)()
+    nph = _lib().oc_profile_read(ms, ln, k)
+    if nph < 0 or nph > k:
+        raise OcError(nph, "oc_profile_read", oc_last_error())
+    return {_lib().oc_profile_phase_name(i).decode(): (ms[i], ln[i]) for i in range(nph)}
+
+
+def oc_launch_count() -> int:
+    return _lib().oc_launch_count()
+
+
+def oc_workspace_release() -> None:
+    _check(_lib().oc_workspace_release(), "oc_workspace_release")
+
+
+def _dev_ptr(t, dtype, name, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def oc_hessian_accumulate(X, H, stream=None):
+    """H += 2 X^T X for bf16 token-major X [n_tok, n] into fp32 H [n, n] (in place)."""
+    import torch
+    n_tok, n = X.shape
+    st = _lib().oc_hessian_accumulate(_dev_ptr(X, torch.bfloat16, "X"), n_tok, n,
+                                   _dev_ptr(H, torch.float32, "H", (n, n)), _stream_handle(stream))
+    _check(st, "oc_hessian_accumulate")
+    return H
+
+
+def oc_qep_correct(W, X, Xhat, alpha, damp, H_opt=None, W_out=None, stream=None):
+    """QEP correction W_out = W + alpha W (X - Xhat)^T Xhat (Xhat^T Xhat + lam I)^-1."""
+    import torch
+    m, n = W.shape
+    n_tok = X.shape[0]
+    if W_out is None:
+        W_out = torch.empty_like(W)
+    hp = _dev_ptr(H_opt, torch.float32, "H_opt", (n, n)) if H_opt is not None else None
+    st = _lib().oc_qep_correct(_dev_ptr(W, torch.float32, "W"), m, n,
+                            _dev_ptr(X, torch.bfloat16, "X", (n_tok, n)),
+                            _dev_ptr(Xhat, torch.bfloat16, "Xhat", (n_tok, n)), n_tok,
+                            float(alpha), float(damp), hp,
+                            _dev_ptr(W_out, torch.float32, "W_out", (m, n)), _stream_handle(stream))
+    _check(st, "oc_qep_correct")
+    return W_out
+
+
+def oc_gptq_quantize(W, H, wbits, groupsize, damp, act_order, codes=None, scales=None,
+                     zeros=None, perm_out=None, stream=None):
+    """GPTQ with per-group asymmetric grids; returns (codes, scales, zeros, perm_out)."""
+    import torch
+    m, n = W.shape
+    G = n if groupsize == -1 else int(groupsize)
+    ng = max(1, n // G)
+    dev = W.device
+    if codes is None:
+        codes = torch.empty(m, n * wbits // 32, dtype=torch.int32, device=dev)
+    if scales is None:
+        scales = torch.empty(m, ng, dtype=torch.float32, device=dev)
+    if zeros is None:
+        zeros = torch.empty(m, ng, dtype=torch.float32, device=dev)
+    pp = _dev_ptr(perm_out, torch.int32, "perm_out", (n,)) if perm_out is not None else None
+    st = _lib().oc_gptq_quantize(_dev_ptr(W, torch.float32, "W"), m, n,
+                              _dev_ptr(H, torch.float32, "H", (n, n)), int(wbits), int(groupsize),
+                              float(damp), 1 if act_order else 0,
+                              _dev_ptr(codes, torch.int32, "codes", (m, n * wbits // 32)),
+                              _dev_ptr(scales, torch.float32, "scales", (m, ng)),
+                              _dev_ptr(zeros, torch.float32, "zeros", (m, ng)), pp,
+                              _stream_handle(stream))
+    _check(st, "oc_gptq_quantize")
+    return codes, scales, zeros, perm_out

@@ -1,0 +1,416 @@
+// C ABI entry points (include/oc.h): argument checks, per-device workspace and
+// status word, and the sequencing of the kernels of each call.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "oc_internal.cuh"
+
+namespace oc {
+
+namespace {
+
+thread_local char g_last_error[768] = "";
+int g_sync_mode = 1;
+std::mutex g_mu;
+
+struct DeviceState {
+  bool init = false;
+  int sm_count = 0;
+  int cc_major = 0, cc_minor = 0;
+  int* status = nullptr;  // device status word
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+};
+DeviceState g_dev[64];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    check_cuda(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q),
+               "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)");
+    if (q != cudaDriverEntryPointSuccess || p == nullptr)
+      fail(OC_ERR_UNSUPPORTED, "driver does not provide cuTensorMapEncodeTiled");
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+DeviceState& device_state(int dev) {
+  if (dev < 0 || dev >= 64) fail(OC_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  DeviceState& d = g_dev[dev];
+  if (!d.init) {
+    check_cuda(cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev), "sm count");
+    check_cuda(cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev), "cc major");
+    check_cuda(cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev), "cc minor");
+    check_cuda(cudaMalloc(&d.status, 256), "cudaMalloc(status)");
+    check_cuda(cudaMemset(d.status, 0, 256), "cudaMemset(status)");
+    d.init = true;
+  }
+  if (d.cc_major != 10 || d.cc_minor != 0)
+    fail(OC_ERR_UNSUPPORTED, "liboc is built for sm_100a; device %d is sm_%d%d", dev, d.cc_major, d.cc_minor);
+  return d;
+}
+
+Ctx make_ctx(void* stream) {
+  int dev = 0;
+  check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
+  DeviceState& d = device_state(dev);
+  Ctx c{};
+  c.stream = static_cast<cudaStream_t>(stream);
+  c.status = d.status;
+  c.sm_count = d.sm_count;
+  c.device = dev;
+  return c;
+}
+
+// Bump allocator over the device workspace (256-byte aligned pieces).
+struct Carve {
+  char* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t count) {
+    off = (off + 255) & ~static_cast<size_t>(255);
+    T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+char* workspace(const Ctx& c, size_t bytes) {
+  DeviceState& d = g_dev[c.device];
+  if (d.ws_bytes < bytes) {
+    if (d.ws) {
+      check_cuda(cudaDeviceSynchronize(), "cudaDeviceSynchronize (workspace grow)");
+      check_cuda(cudaFree(d.ws), "cudaFree(workspace)");
+      d.ws = nullptr;
+      d.ws_bytes = 0;
+    }
+    const size_t want = bytes + (bytes >> 4);
+    if (cudaMalloc(&d.ws, want) != cudaSuccess) {
+      cudaGetLastError();
+      d.ws = nullptr;
+      fail(OC_ERR_OOM, "could not allocate a %zu-byte workspace", want);
+    }
+    d.ws_bytes = want;
+  }
+  return static_cast<char*>(d.ws);
+}
+
+int finish(const Ctx& c) {
+  if (!g_sync_mode) return OC_OK;
+  check_cuda(cudaStreamSynchronize(c.stream), "cudaStreamSynchronize");
+  int st = 0;
+  check_cuda(cudaMemcpy(&st, c.status, sizeof(int), cudaMemcpyDeviceToHost), "read status");
+  if (st != 0) {
+    check_cuda(cudaMemset(c.status, 0, sizeof(int)), "reset status");
+    snprintf(g_last_error, sizeof(g_last_error), "device reported %s", oc_status_string(st));
+  }
+  return st;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <class F>
+int guarded(F&& f) {
+  try {
+    g_last_error[0] = '\0';
+    std::lock_guard<std::mutex> lock(g_mu);
+    return f();
+  } catch (const Failure& e) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s", e.msg);
+    return e.status;
+  } catch (const std::bad_alloc&) {
+    snprintf(g_last_error, sizeof(g_last_error), "host allocation failed");
+    return OC_ERR_OOM;
+  }
+}
+
+}  // namespace
+
+void fail(int status, const char* fmt, ...) {
+  Failure f{};
+  f.status = status;
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(f.msg, sizeof(f.msg), fmt, ap);
+  va_end(ap);
+  throw f;
+}
+
+void check_cuda(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) fail(OC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+void check_launch(const char* kernel) {
+  count_launch();
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) fail(OC_ERR_CUDA, "launch of %s failed: %s", kernel, cudaGetErrorString(e));
+}
+
+CUtensorMap make_tmap_2d(const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t rows, uint64_t cols,
+                         uint64_t ld, uint32_t box_rows, uint32_t box_cols, Swz swz) {
+  if (!aligned16(base)) fail(OC_ERR_INVALID_ARG, "TMA base address must be 16-byte aligned");
+  if ((ld * elem_bytes) % 16) fail(OC_ERR_INVALID_ARG, "TMA row pitch must be a multiple of 16 bytes");
+  CUtensorMap m;
+  std::memset(&m, 0, sizeof(m));
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {ld * static_cast<uint64_t>(elem_bytes)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode_fn()(&m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                                 CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 swz == Swz::B128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) fail(OC_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return m;
+}
+
+}  // namespace oc
+
+using namespace oc;
+
+extern "C" {
+
+const char* oc_status_string(int status) {
+  switch (status) {
+    case OC_OK: return "OC_OK";
+    case OC_ERR_INVALID_ARG: return "OC_ERR_INVALID_ARG";
+    case OC_ERR_UNSUPPORTED: return "OC_ERR_UNSUPPORTED";
+    case OC_ERR_NOT_SPD: return "OC_ERR_NOT_SPD";
+    case OC_ERR_NONFINITE: return "OC_ERR_NONFINITE";
+    case OC_ERR_TIMEOUT: return "OC_ERR_TIMEOUT";
+    case OC_ERR_CUDA: return "OC_ERR_CUDA";
+    case OC_ERR_OOM: return "OC_ERR_OOM";
+    default: return "OC_ERR_UNKNOWN";
+  }
+}
+
+const char* oc_last_error(void) { return g_last_error; }
+
+int oc_version(void) { return 100; }
+
+void oc_set_sync(int sync) { g_sync_mode = sync ? 1 : 0; }
+
+int oc_stream_status(void* stream) {
+  return guarded([&]() -> int {
+    Ctx c = make_ctx(stream);
+    check_cuda(cudaStreamSynchronize(c.stream), "cudaStreamSynchronize");
+    int st = 0;
+    check_cuda(cudaMemcpy(&st, c.status, sizeof(int), cudaMemcpyDeviceToHost), "read status");
+    if (st != 0) check_cuda(cudaMemset(c.status, 0, sizeof(int)), "reset status");
+    return st;
+  });
+}
+
+int oc_profile_enable(int on) {
+  return guarded([&]() -> int {
+    profile_enable(on != 0);
+    return OC_OK;
+  });
+}
+
+int oc_profile_read(double* ms, int64_t* launches, int max_phases) {
+  return guarded([&]() -> int { return profile_read(ms, launches, max_phases); });
+}
+
+const char* oc_profile_phase_name(int phase) { return phase_name(phase); }
+
+int64_t oc_launch_count(void) { return launch_count(); }
+
+int oc_workspace_release(void) {
+  return guarded([&]() -> int {
+    int dev = 0;
+    check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev >= 0 && dev < 64 && g_dev[dev].ws) {
+      check_cuda(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+      check_cuda(cudaFree(g_dev[dev].ws), "cudaFree(workspace)");
+      g_dev[dev].ws = nullptr;
+      g_dev[dev].ws_bytes = 0;
+    }
+    return OC_OK;
+  });
+}
+
+int oc_hessian_accumulate(const void* X, int64_t n_tok, int64_t n, float* H, void* stream) {
+  return guarded([&]() -> int {
+    if (!H) fail(OC_ERR_INVALID_ARG, "H must be non-null");
+    if (n < 64 || n % 64) fail(OC_ERR_INVALID_ARG, "n must be a positive multiple of 64 (got %lld)", (long long)n);
+    if (n_tok < 0) fail(OC_ERR_INVALID_ARG, "n_tok must be >= 0");
+    if (n_tok == 0) return OC_OK;  // nothing to add (X may be NULL)
+    if (!X) fail(OC_ERR_INVALID_ARG, "X must be non-null");
+    if (n_tok > (int64_t(1) << 31) - 64) fail(OC_ERR_INVALID_ARG, "n_tok too large for one call; split it");
+    if (!aligned16(X) || !aligned16(H)) fail(OC_ERR_INVALID_ARG, "X and H must be 16-byte aligned");
+    Ctx c = make_ctx(stream);
+    {
+      PhaseScope ps(c, kPhHessian);
+      launch_atb_bf16(c, X, X, n_tok, n, n, 2.0f, H, n, true);
+      launch_mirror_upper(c, H, n);
+    }
+    return finish(c);
+  });
+}
+
+int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const void* Xhat, int64_t n_tok,
+                   float alpha, float damp, const float* H_opt, float* W_out, void* stream) {
+  return guarded([&]() -> int {
+    if (!W || !X || !Xhat || !W_out) fail(OC_ERR_INVALID_ARG, "W, X, Xhat, W_out must be non-null");
+    if (n < 64 || n % 64) fail(OC_ERR_INVALID_ARG, "n must be a positive multiple of 64");
+    if (n > 49152) fail(OC_ERR_INVALID_ARG, "n above 49152 is not supported");
+    if (m < 1) fail(OC_ERR_INVALID_ARG, "m must be >= 1");
+    if (n_tok < 1 || n_tok > (int64_t(1) << 31) - 64) fail(OC_ERR_INVALID_ARG, "n_tok out of range");
+    if (!(alpha == alpha) || alpha > 3.4e38f || alpha < -3.4e38f) fail(OC_ERR_INVALID_ARG, "alpha must be finite");
+    if (!(damp >= 0.f) || damp > 3.4e38f) fail(OC_ERR_INVALID_ARG, "damp must be finite and >= 0");
+    if (!aligned16(X) || !aligned16(Xhat) || (H_opt && !aligned16(H_opt)))
+      fail(OC_ERR_INVALID_ARG, "X, Xhat, H_opt must be 16-byte aligned");
+    Ctx c = make_ctx(stream);
+    const size_t nn = static_cast<size_t>(n) * n, mn = static_cast<size_t>(m) * n;
+    if (alpha == 0.f) {
+      if (W_out != W) launch_copy_f32(c, W, W_out, static_cast<int64_t>(mn));
+      return finish(c);
+    }
+    Carve sizing{nullptr};
+    sizing.take<float>(nn);                       // D -> M -> U
+    if (!H_opt) sizing.take<float>(nn);           // Hs
+    sizing.take<float>(nn);                       // X (inverse factor of the reversed matrix)
+    sizing.take<float>(nn / 2 + 4096);            // recursion scratch
+    sizing.take<float>(mn);                       // G
+    sizing.take<float>(mn);                       // T
+    sizing.take<DiagStats>(1);
+    Carve cv{workspace(c, sizing.off + 256)};
+    float* D = cv.take<float>(nn);
+    float* Hs = H_opt ? nullptr : cv.take<float>(nn);
+    float* Xi = cv.take<float>(nn);
+    float* scratch = cv.take<float>(nn / 2 + 4096);
+    float* G = cv.take<float>(mn);
+    float* T = cv.take<float>(mn);
+    DiagStats* stats = cv.take<DiagStats>(1);
+
+    // d = X^T Xhat - Xhat^T Xhat  (the second term from H = 2 Xhat^T Xhat)
+    const float* Hp = H_opt;
+    if (!H_opt) {
+      PhaseScope ps(c, kPhQepSyrk);
+      check_cuda(cudaMemsetAsync(Hs, 0, nn * sizeof(float), c.stream), "memset Hs");
+      launch_atb_bf16(c, Xhat, Xhat, n_tok, n, n, 2.0f, Hs, n, true);
+      launch_mirror_upper(c, Hs, n);
+      Hp = Hs;
+    }
+    {
+      PhaseScope ps(c, kPhQepCross);
+      check_cuda(cudaMemsetAsync(D, 0, nn * sizeof(float), c.stream), "memset D");
+      launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false);
+      launch_sub_half(c, D, Hp, n);
+    }
+    {
+      // G = W d
+      PhaseScope ps(c, kPhQepWDelta);
+      gemm_f32(c, false, false, m, n, n, 1.f, W, n, D, n, 0.f, G, n, kANone);
+    }
+    {
+      // 2A = Hp + damp mean(diag Hp) I = R R^T;  U = R^-1 upper, A^-1 = 2 U^T U
+      PhaseScope ps(c, kPhFactor);
+      launch_diag_stats(c, Hp, n, damp, 1.0f, false, stats, nullptr);
+      launch_build_reversed(c, Hp, n, nullptr, stats, 1.0f, false, D);
+      factor_inverse_upper(c, D, Xi, scratch, D, n);
+    }
+    {
+      // W_out = W + alpha G A^-1 = W + 2 alpha (G U^T) U
+      PhaseScope ps(c, kPhQepApply);
+      const float* U = D;
+      gemm_f32(c, false, true, m, n, n, 1.f, G, n, U, n, 0.f, T, n, kBLower);
+      if (W_out != W) launch_copy_f32(c, W, W_out, static_cast<int64_t>(mn));
+      gemm_f32(c, false, false, m, n, n, 2.f * alpha, T, n, U, n, 1.f, W_out, n, kBUpper);
+    }
+    return finish(c);
+  });
+}
+
+int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int wbits, int groupsize, float damp,
+                     int act_order, uint32_t* codes, float* scales, float* zeros, int32_t* perm_out,
+                     void* stream) {
+  return guarded([&]() -> int {
+    if (!W || !H || !codes || !scales || !zeros) fail(OC_ERR_INVALID_ARG, "W, H, codes, scales, zeros must be non-null");
+    if (n < 64 || n % 64) fail(OC_ERR_INVALID_ARG, "n must be a positive multiple of 64");
+    if (n > 49152) fail(OC_ERR_INVALID_ARG, "n above 49152 is not supported");
+    if (m < 1) fail(OC_ERR_INVALID_ARG, "m must be >= 1");
+    if (wbits < 2 || wbits > 4) fail(OC_ERR_INVALID_ARG, "wbits must be 2, 3 or 4");
+    if (act_order != 0 && act_order != 1) fail(OC_ERR_INVALID_ARG, "act_order must be 0 or 1");
+    if (!(damp >= 0.f) || damp > 3.4e38f) fail(OC_ERR_INVALID_ARG, "damp must be finite and >= 0");
+    const int64_t G = (groupsize == -1) ? n : groupsize;
+    if (G < 4 || n % G) fail(OC_ERR_INVALID_ARG, "groupsize must divide n (or be -1)");
+    const bool pow2_small = G <= 128 && (G & (G - 1)) == 0;
+    if (!(G == n || pow2_small || G % 128 == 0))
+      fail(OC_ERR_INVALID_ARG, "groupsize must be a power of two <= 128, a multiple of 128, or -1");
+    if (!aligned16(codes) || !aligned16(W)) fail(OC_ERR_INVALID_ARG, "W and codes must be 16-byte aligned");
+    Ctx c = make_ctx(stream);
+    const size_t nn = static_cast<size_t>(n) * n, mn = static_cast<size_t>(m) * n;
+    Carve sizing{nullptr};
+    sizing.take<float>(nn);            // M -> U
+    sizing.take<float>(nn);            // X
+    sizing.take<float>(nn / 2 + 4096); // scratch
+    sizing.take<float>(mn);            // Wp
+    sizing.take<unsigned char>(mn);    // codes8
+    sizing.take<float>(static_cast<size_t>(m) * 128);  // Err
+    sizing.take<int32_t>(2 * static_cast<size_t>(n));  // perm | inverse
+    sizing.take<unsigned char>(n);     // dead
+    sizing.take<DiagStats>(1);
+    Carve cv{workspace(c, sizing.off + 256)};
+    float* M = cv.take<float>(nn);
+    float* Xi = cv.take<float>(nn);
+    float* scratch = cv.take<float>(nn / 2 + 4096);
+    float* Wp = cv.take<float>(mn);
+    unsigned char* codes8 = cv.take<unsigned char>(mn);
+    float* Err = cv.take<float>(static_cast<size_t>(m) * 128);
+    int32_t* perm = cv.take<int32_t>(2 * static_cast<size_t>(n));
+    unsigned char* dead = cv.take<unsigned char>(n);
+    DiagStats* stats = cv.take<DiagStats>(1);
+
+    {
+      PhaseScope ps(c, kPhFactor);
+      launch_diag_stats(c, H, n, damp, 1.0f, true, stats, dead);
+      if (act_order) launch_act_order_perm(c, H, n, perm);
+      else launch_identity_perm(c, n, perm);
+      launch_build_reversed(c, H, n, perm, stats, 1.0f, true, M);
+      factor_inverse_upper(c, M, Xi, scratch, M, n);
+    }
+    const float* U = M;
+    {
+      PhaseScope ps(c, kPhGptqPrep);
+      launch_permute_w(c, W, m, n, perm, dead, Wp);
+      if (act_order) launch_static_grid(c, W, m, n, static_cast<int>(G), wbits, dead, scales, zeros);
+    }
+    for (int64_t j1 = 0; j1 < n; j1 += 128) {
+      const int64_t bw = std::min<int64_t>(128, n - j1);
+      const int64_t j2 = j1 + bw;
+      {
+        PhaseScope ps(c, kPhGptqSweep);
+        launch_sweep_block(c, Wp, m, n, U, j1, static_cast<int>(G), wbits, act_order != 0, perm, scales, zeros,
+                           codes8, Err);
+      }
+      if (j2 < n) {
+        PhaseScope ps(c, kPhGptqTrailing);
+        gemm_f32(c, false, false, m, n - j2, bw, -1.f, Err, 128, U + j1 * n + j2, n, 1.f, Wp + j2, n, kANone);
+      }
+    }
+    {
+      PhaseScope ps(c, kPhGptqPack);
+      launch_pack(c, codes8, m, n, wbits, perm, codes);
+    }
+    if (perm_out)
+      check_cuda(cudaMemcpyAsync(perm_out, perm, static_cast<size_t>(n) * sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                                 c.stream),
+                 "copy perm");
+    return finish(c);
+  });
+}
+
+}  // extern "C"

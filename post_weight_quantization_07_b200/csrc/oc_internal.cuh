@@ -1,0 +1,158 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/oc.h"
+
+namespace oc {
+
+// Device-side error codes recorded in the status word (same values as oc_status).
+enum DevErr : int {
+  kDevOk = 0,
+  kDevNotSpd = OC_ERR_NOT_SPD,
+  kDevNonfinite = OC_ERR_NONFINITE,
+  kDevTimeout = OC_ERR_TIMEOUT,
+};
+
+// Record the first device-side error (later ones are dropped).
+__device__ __forceinline__ void record_error(int* status, int code) {
+  if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+// Per-call context handed to the internal launchers.
+struct Ctx {
+  cudaStream_t stream;
+  int* status;      // device status word
+  int sm_count;
+  int device;
+};
+
+// Host-side failure carrying a status and a message (converted to the C ABI
+// return value at the boundary).
+struct Failure {
+  int status;
+  char msg[512];
+};
+[[noreturn]] void fail(int status, const char* fmt, ...);
+void check_cuda(cudaError_t e, const char* what);
+void check_launch(const char* kernel);
+
+// ------------------------------------------------------------------ profiling
+enum Phase : int {
+  kPhHessian = 0,   // oc_hessian_accumulate: tensor-core SYRK + mirror
+  kPhQepCross,      // X^T Xhat on the tensor cores, minus Xhat^T Xhat
+  kPhQepSyrk,       // Xhat^T Xhat when no H is supplied
+  kPhQepWDelta,     // G = W d
+  kPhFactor,        // dampening, reversal, blocked Cholesky + inverse, reversal
+  kPhQepApply,      // W + 2 alpha (G U^T) U
+  kPhGptqPrep,      // act_order order, permutation of W, static grid
+  kPhGptqSweep,     // 128-column block sweeps
+  kPhGptqTrailing,  // trailing updates of later columns
+  kPhGptqPack,      // inverse permutation + bit packing
+  kNumPhases
+};
+
+void count_launch();
+int64_t launch_count();
+void profile_enable(bool on);
+int profile_read(double* ms, int64_t* launches, int max_phases);
+const char* phase_name(int p);
+
+// Records a CUDA event pair around its lifetime on the call's stream when
+// profiling is enabled (no-op otherwise).
+class PhaseScope {
+ public:
+  PhaseScope(const struct Ctx& c, Phase p);
+  ~PhaseScope();
+  PhaseScope(const PhaseScope&) = delete;
+  PhaseScope& operator=(const PhaseScope&) = delete;
+
+ private:
+  cudaStream_t stream_;
+  Phase phase_;
+  cudaEvent_t a_ = nullptr;
+  int64_t l0_ = 0;
+  bool active_ = false;
+};
+
+// TMA descriptor for a row-major 2-D array [rows x cols] of `elem_bytes`
+// elements with leading dimension `ld` (elements), box [box_rows x box_cols].
+enum class Swz { None, B128 };
+CUtensorMap make_tmap_2d(const void* base, CUtensorMapDataType dt, int elem_bytes,
+                         uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows,
+                         uint32_t box_cols, Swz swz);
+
+// ------------------------------------------------------------------ kernels
+
+// C[i][j] += alpha * sum_t A[t][i] * B[t][j] with A, B bf16 token-major
+// [n_tok x M] and [n_tok x N]; C fp32 [M x N] (ldc).  upper_only: A == B and
+// only tiles touching the upper triangle are computed (the caller mirrors).
+void launch_atb_bf16(const Ctx& c, const void* A, const void* B, int64_t n_tok, int64_t M,
+                     int64_t N, float alpha, float* C, int64_t ldc, bool upper_only);
+
+// Mirror the upper triangle of an n x n matrix into its lower triangle.
+void launch_mirror_upper(const Ctx& c, float* H, int64_t n);
+
+// Flags for gemm_f32: triangular structure of op(A)/op(B) (zeros skipped) and
+// C tiles wholly above the diagonal skipped.
+enum GemmFlags : unsigned {
+  kANone = 0,
+  kALower = 1u << 0,
+  kAUpper = 1u << 1,
+  kBLower = 1u << 2,
+  kBUpper = 1u << 3,
+  kCLowerOnly = 1u << 4,
+};
+
+// C = beta*C + alpha*op(A)*op(B), fp32, row-major, op = transpose when tX.
+void gemm_f32(const Ctx& c, bool tA, bool tB, int64_t M, int64_t N, int64_t K, float alpha,
+              const float* A, int64_t lda, const float* B, int64_t ldb, float beta, float* C,
+              int64_t ldc, unsigned flags);
+
+// U = upper Cholesky factor of (H_prepared)^-1, where H_prepared is formed by
+// `launch_build_reversed` into M (consumed).  Scratch must hold n*n/2 + 4096
+// floats.  X receives L^-1 of the reversed matrix (lower), U its reversal.
+void factor_inverse_upper(const Ctx& c, float* M, float* X, float* scratch, float* U,
+                          int64_t n);
+
+// M[a][b] = Hfix[p(n-1-a)][p(n-1-b)] + lam*[a==b] where Hfix has dead
+// diagonal entries set to 1 (when fix_dead), p = perm (identity if null) and
+// lam = damp * mean(diag Hfix) (computed on device into stats).
+struct DiagStats {
+  float lam;
+  float mean_diag;
+  int n_dead;
+  int nonfinite;
+};
+void launch_diag_stats(const Ctx& c, const float* H, int64_t n, float damp, float hscale,
+                       bool fix_dead, DiagStats* stats, unsigned char* dead);
+void launch_act_order_perm(const Ctx& c, const float* H, int64_t n, int32_t* perm);
+void launch_identity_perm(const Ctx& c, int64_t n, int32_t* perm);
+void launch_build_reversed(const Ctx& c, const float* H, int64_t n, const int32_t* perm,
+                           const DiagStats* stats, float hscale, bool fix_dead, float* M);
+
+// GPTQ pieces.
+void launch_permute_w(const Ctx& c, const float* W, int64_t m, int64_t n, const int32_t* perm,
+                      const unsigned char* dead, float* Wp);
+void launch_static_grid(const Ctx& c, const float* W, int64_t m, int64_t n, int G, int wbits,
+                        const unsigned char* dead, float* scales, float* zeros);
+void launch_sweep_block(const Ctx& c, float* Wp, int64_t m, int64_t n, const float* U,
+                        int64_t j1, int G, int wbits, bool static_groups, const int32_t* perm,
+                        float* scales, float* zeros, unsigned char* codes8, float* Err);
+// Packs codes8 (processing order) into the original-order bitstream; perm2
+// holds the processing order in its first n entries and receives the inverse
+// permutation in the next n.
+void launch_pack(const Ctx& c, const unsigned char* codes8, int64_t m, int64_t n, int wbits,
+                 int32_t* perm2, uint32_t* codes);
+
+// QEP pieces.
+void launch_sub_half(const Ctx& c, float* D, const float* H, int64_t n);  // D -= H/2
+void launch_copy_f32(const Ctx& c, const float* src, float* dst, int64_t count);
+void launch_fill_f32(const Ctx& c, float* dst, int64_t count, float v);
+void launch_check_finite(const Ctx& c, const float* x, int64_t count);
+
+}  // namespace oc

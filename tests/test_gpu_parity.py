@@ -1,0 +1,251 @@
+"""GPU parity: the CUDA path (called through the C ABI) against the float64
+oracle on the same seeded inputs.
+
+Tolerances (the quantisation workload's stated bars):
+  Hessian           relative Frobenius error <= 1e-4 (oracle fed the same bf16 inputs);
+  codes             >= 99.9% identical, and every mismatch, replayed with the
+                    candidate's earlier decisions forced in, lies within 1e-3 of a
+                    rounding boundary (in units of the scale).  Identity is counted
+                    on the integer levels q - zero: a zero decided at a rounding
+                    boundary shifts every code of its group by one and leaves each
+                    dequantised weight scale * (q - zero) unchanged;
+  scales / zeros    relative error <= 1e-5 (zeros: equal unless -min/scale sits
+                    within 1e-3 of a rounding boundary);
+  layer error       ||(W - Q) X^T||_F within 1% of the oracle's.
+QEP output: max |W'_gpu - W'_oracle| <= 1e-5 * max |W| (derived in the design
+notes from the fp32 arithmetic of the path).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from synthetic import CONFIGS, make_layer_host, random_layer_host
+
+torch = pytest.importorskip("torch")
+oc = pytest.importorskip("post_weight_quantization_07_b200")
+
+pytestmark = pytest.mark.gpu
+
+H_TOL = 1e-4
+SCALE_TOL = 1e-5
+CODE_FRAC = 0.999
+BOUNDARY = 1e-3
+QEP_TOL = 1e-5
+
+
+def dev(a, dtype=torch.float32):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device="cuda", dtype=dtype)
+
+
+def bf16_dev(a):
+    # values are already bf16-representable (synthetic rounds them): exact cast
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to("cuda").to(torch.bfloat16)
+
+
+def rel_fro(a, b):
+    return float(np.linalg.norm(np.asarray(a, np.float64) - b) / np.linalg.norm(b))
+
+
+def gpu_hessian(xhat_np, H0=None):
+    n = xhat_np.shape[1]
+    H = dev(np.zeros((n, n)) if H0 is None else H0)
+    oc.oc_hessian_accumulate(bf16_dev(xhat_np), H)
+    torch.cuda.synchronize()
+    return H.cpu().numpy()
+
+
+# ----------------------------------------------------------------------------- Hessian
+
+@pytest.mark.parametrize("n,n_tok", [(64, 100), (256, 1000), (384, 777), (512, 2048), (640, 4096 + 33)])
+def test_hessian_matches_oracle(n, n_tok):
+    L = random_layer_host(8, n, n_tok, seed=100 + n)
+    Hg = gpu_hessian(L["Xhat"])
+    Ho = oracle.hessian(L["Xhat"])
+    assert rel_fro(Hg, Ho) <= H_TOL
+    assert np.array_equal(Hg, Hg.T)
+
+
+def test_hessian_accumulates_and_ignores_empty():
+    L = random_layer_host(8, 256, 1500, seed=7)
+    H1 = gpu_hessian(L["Xhat"][:700])
+    H2 = gpu_hessian(L["Xhat"][700:], H0=H1)
+    Ho = oracle.hessian(L["Xhat"])
+    assert rel_fro(H2, Ho) <= H_TOL
+    H = dev(H2)
+    oc.oc_hessian_accumulate(torch.empty(0, 256, dtype=torch.bfloat16, device="cuda"), H)
+    assert np.array_equal(H.cpu().numpy(), H2)
+
+
+# ----------------------------------------------------------------------------- QEP
+
+def _qep_case(n=256, m=96, n_tok=3000, seed=11):
+    L = random_layer_host(m, n, n_tok, seed=seed)
+    return L["W"], L["X"], L["Xhat"]
+
+
+@pytest.mark.parametrize("use_h", [False, True])
+@pytest.mark.parametrize("shape", [(96, 256, 3000), (512, 512, 2048), (130, 384, 1111)])
+def test_qep_matches_oracle(use_h, shape):
+    m, n, n_tok = shape
+    W, X, Xh = _qep_case(n=n, m=m, n_tok=n_tok, seed=m + n)
+    alpha, damp = 0.5, 0.01
+    Ho = oracle.hessian(Xh)
+    Wo = oracle.qep_correct(W, X, Xh, alpha, damp, H=Ho)
+    Hg = dev(gpu_hessian(Xh)) if use_h else None
+    Wg = oc.oc_qep_correct(dev(W), bf16_dev(X), bf16_dev(Xh), alpha, damp, H_opt=Hg).cpu().numpy()
+    err = np.abs(Wg - Wo).max()
+    corr = np.abs(Wo - W).max()
+    assert err <= QEP_TOL * np.abs(W).max(), (err, corr)
+    # the correction itself is reproduced to a small fraction of its size
+    assert np.abs((Wg - W) - (Wo - W)).max() <= 2e-3 * corr
+
+
+def test_qep_alpha_zero_is_identity_bitwise():
+    W, X, Xh = _qep_case()
+    Wd = dev(W)
+    out = oc.oc_qep_correct(Wd, bf16_dev(X), bf16_dev(Xh), 0.0, 0.01)
+    assert torch.equal(out, Wd)
+    same = oc.oc_qep_correct(Wd, bf16_dev(X), bf16_dev(Xh), 0.0, 0.01, W_out=Wd)
+    assert torch.equal(same, dev(W))
+
+
+def test_qep_identical_inputs_leave_w():
+    W, X, _ = _qep_case()
+    out = oc.oc_qep_correct(dev(W), bf16_dev(X), bf16_dev(X), 0.5, 0.01).cpu().numpy()
+    assert np.abs(out - W).max() <= 1e-6 * np.abs(W).max()
+
+
+def test_qep_in_place():
+    W, X, Xh = _qep_case()
+    Wd = dev(W)
+    ref = oc.oc_qep_correct(Wd, bf16_dev(X), bf16_dev(Xh), 0.5, 0.01).clone()
+    oc.oc_qep_correct(Wd, bf16_dev(X), bf16_dev(Xh), 0.5, 0.01, W_out=Wd)
+    assert torch.allclose(Wd, ref, rtol=0, atol=1e-7)
+
+
+# ----------------------------------------------------------------------------- GPTQ
+
+def gpu_gptq(W, H, wbits, G, damp, act_order):
+    m, n = W.shape
+    perm = torch.empty(n, dtype=torch.int32, device="cuda")
+    codes, scales, zeros, _ = oc.oc_gptq_quantize(dev(W), dev(H), wbits, G, damp, act_order,
+                                                  perm_out=perm)
+    torch.cuda.synchronize()
+    words = codes.cpu().numpy().view(np.uint32)
+    return (oracle.unpack_codes(words, wbits, n), scales.cpu().numpy(), zeros.cpu().numpy(),
+            perm.cpu().numpy(), words)
+
+
+def level_identity(codes_a, zeros_a, codes_b, zeros_b, G):
+    n = codes_a.shape[1]
+    G = n if G == -1 else G
+    la = codes_a - np.repeat(zeros_a, G, axis=1)
+    lb = codes_b - np.repeat(zeros_b, G, axis=1)
+    return float(np.mean(la == lb))
+
+
+def check_gptq(W, H, wbits, G, damp, act_order, gpu=None):
+    codes, scales, zeros, perm, words = gpu if gpu is not None else gpu_gptq(W, H, wbits, G, damp, act_order)
+    ref = oracle.gptq_quantize(W, H, wbits, G, damp, act_order)
+    assert np.array_equal(perm, ref["perm"])
+    ident = level_identity(codes, zeros, ref["codes"], ref["zeros"], G)
+    st = oracle.teacher_forced_check(W, H, wbits, G, damp, act_order, codes, scales, zeros, perm=perm)
+    assert ident >= CODE_FRAC, (ident, st)
+    assert st["n_bad"] == 0, st
+    assert st["scale_max_rel"] <= SCALE_TOL, st
+    assert st["zero_bad"] == 0, st
+    assert np.array_equal(words, ref["packed"]) or ident < 1.0
+    return ident, st
+
+
+@pytest.mark.parametrize("m,n,wbits,G,act", [
+    (512, 512, 4, 128, False),   # the 512 x 512 workload's settings
+    (200, 384, 3, 64, True),
+    (96, 320, 2, 32, False),     # ragged last block (64 columns)
+    (64, 512, 4, 256, False),    # group wider than a block
+    (64, 256, 3, -1, True),
+    (33, 192, 4, -1, False),     # one group of 192 columns across two blocks
+    (7, 128, 2, 4, False),       # tiny groups, fewer rows than a CTA's warps
+])
+def test_gptq_matches_oracle(m, n, wbits, G, act):
+    L = random_layer_host(m, n, max(2 * n, 512), seed=1000 + m + n)
+    H = oracle.hessian(L["Xhat"]).astype(np.float32).astype(np.float64)
+    check_gptq(L["W"].astype(np.float64), H, wbits, G, 0.01, act)
+
+
+def test_gptq_identity_hessian_is_rtn():
+    r = np.random.default_rng(3)
+    W = (r.standard_normal((64, 256)) * 0.02).astype(np.float32).astype(np.float64)
+    H = np.eye(256)
+    codes, scales, zeros, perm, _ = gpu_gptq(W, H, 4, 64, 0.01, False)
+    ref = oracle.gptq_quantize(W, H, 4, 64, 0.01, False)
+    assert np.array_equal(codes, ref["codes"])
+
+
+def test_gptq_dead_columns():
+    L = random_layer_host(48, 256, 1024, seed=21)
+    x = L["Xhat"].copy()
+    x[:, [3, 100, 255]] = 0.0
+    H = oracle.hessian(x).astype(np.float32).astype(np.float64)
+    for act in (False, True):
+        check_gptq(L["W"].astype(np.float64), H, 4, 64, 0.01, act)
+
+
+def test_gptq_not_spd_reports_error():
+    n = 128
+    r = np.random.default_rng(5)
+    Q, _ = np.linalg.qr(r.standard_normal((n, n)))
+    ev = np.linspace(1.0, 2.0, n)
+    ev[17] = -0.5
+    H = (Q * ev) @ Q.T
+    W = r.standard_normal((16, n)) * 0.02
+    with pytest.raises(oc.OcError) as e:
+        oc.oc_gptq_quantize(dev(W), dev(H), 4, 128, 0.0, False)
+    assert e.value.status == oc.OC_ERR_NOT_SPD
+    # the library stays usable afterwards
+    check_gptq(W, np.eye(n) * 2.0, 4, 128, 0.0, False)
+
+
+def test_gptq_nonfinite_reports_error():
+    n = 128
+    H = np.eye(n)
+    H[5, 5] = np.nan
+    W = np.zeros((8, n))
+    with pytest.raises(oc.OcError) as e:
+        oc.oc_gptq_quantize(dev(W), dev(H), 4, 128, 0.01, False)
+    assert e.value.status == oc.OC_ERR_NONFINITE
+
+
+# ----------------------------------------------------------------------------- end to end
+
+def test_end_to_end_512_workload():
+    spec = CONFIGS["c1_512"]
+    L = make_layer_host(spec)
+    W, X, Xh = L["W"].astype(np.float64), L["X"], L["Xhat"]
+    # oracle
+    Ho = oracle.hessian(Xh)
+    Wpo = oracle.qep_correct(W, X, Xh, spec.alpha, spec.damp, H=Ho)
+    ref = oracle.gptq_quantize(Wpo, Ho, spec.wbits, spec.groupsize, spec.damp, spec.act_order)
+    # CUDA path
+    Hg = dev(np.zeros((spec.d_in, spec.d_in)))
+    Xd, Xhd = bf16_dev(X), bf16_dev(Xh)
+    oc.oc_hessian_accumulate(Xhd, Hg)
+    Wp = oc.oc_qep_correct(dev(W), Xd, Xhd, spec.alpha, spec.damp, H_opt=Hg)
+    perm = torch.empty(spec.d_in, dtype=torch.int32, device="cuda")
+    codes, scales, zeros, _ = oc.oc_gptq_quantize(Wp, Hg, spec.wbits, spec.groupsize, spec.damp,
+                                                  spec.act_order, perm_out=perm)
+    torch.cuda.synchronize()
+    assert rel_fro(Hg.cpu().numpy(), Ho) <= H_TOL
+    cg = oracle.unpack_codes(codes.cpu().numpy().view(np.uint32), spec.wbits, spec.d_in)
+    sg, zg = scales.cpu().numpy(), zeros.cpu().numpy()
+    ident = level_identity(cg, zg, ref["codes"], ref["zeros"], spec.groupsize)
+    assert ident >= CODE_FRAC
+    st = oracle.teacher_forced_check(Wpo, Ho, spec.wbits, spec.groupsize, spec.damp,
+                                     spec.act_order, cg, sg, zg, perm=perm.cpu().numpy())
+    assert st["n_bad"] == 0 and st["zero_bad"] == 0, st
+    assert st["scale_max_rel"] <= SCALE_TOL, st
+    G = spec.groupsize
+    deq = np.repeat(sg, G, axis=1) * (cg - np.repeat(zg, G, axis=1))
+    eg = oracle.layer_errors(W, deq, X, Xh)["e_lit"]
+    eo = oracle.layer_errors(W, ref["deq"], X, Xh)["e_lit"]
+    assert abs(eg - eo) <= 0.01 * eo
