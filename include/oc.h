@@ -180,6 +180,38 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
                      int groupsize, float damp, int act_order, uint32_t* codes,
                      float* scales, float* zeros, int32_t* perm_out, void* stream);
 
+/*
+ * Allocation-free GPTQ (no counterpart in the paper: an addition for callers of
+ * this library).  Some callers cannot have a library allocate device memory on
+ * its own -- e.g. a process whose memory is entirely reserved for its own
+ * caching allocator at start-up, or a service held to a fixed, pre-reserved
+ * budget -- because the workspace that oc_gptq_quantize grows with cudaMalloc
+ * (and the device-wide synchronisation of the cudaFree before a regrowth)
+ * would fail or stall there.  This entry point computes exactly what
+ * oc_gptq_quantize computes, with the same arguments, but takes every byte of
+ * scratch from one array built into the library (6 MiB per GPU, held by every
+ * GPU that loads the library until the process exits) and never calls
+ * cudaMalloc, cudaFree or any other allocating routine.  The caller still
+ * passes all inputs and outputs.
+ *   - Size limit: the layer must fit the 6 MiB scratch (about
+ *     10 n^2 + m (5 n + 512) bytes), e.g. n = 512 with m <= 1024, or n = 256
+ *     with m <= 3072; larger requests return OC_ERR_INVALID_ARG with the bytes
+ *     needed in oc_last_error().
+ *   - The first call on a device looks up the array's device address on that
+ *     device (the device must be current); make that first call before any
+ *     stream capture begins.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents (each call clears what must start at zero).  Calls that
+ *     overlap on the GPU -- on different streams or from different threads --
+ *     race on it and must not be issued.
+ *   - Always synchronous: the call waits for its stream and returns the
+ *     device-side status (OC_ERR_NOT_SPD, OC_ERR_NONFINITE, ...), whatever
+ *     oc_set_sync() says.
+ */
+int oc_gptq_quantize_noalloc(const float* W, int64_t m, int64_t n, const float* H, int wbits,
+                             int groupsize, float damp, int act_order, uint32_t* codes,
+                             float* scales, float* zeros, int32_t* perm_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -147,6 +147,8 @@ void fail(int status, const char* fmt, ...) {
   throw f;
 }
 
+void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
 void check_cuda(cudaError_t e, const char* what) {
   if (e != cudaSuccess) fail(OC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }

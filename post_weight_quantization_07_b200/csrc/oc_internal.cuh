@@ -39,6 +39,7 @@ struct Failure {
 };
 [[noreturn]] void fail(int status, const char* fmt, ...);
 void check_cuda(cudaError_t e, const char* what);
+void set_last_error(const char* msg);  // text returned by oc_last_error() on this thread
 void check_launch(const char* kernel);
 
 // ------------------------------------------------------------------ profiling
