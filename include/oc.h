@@ -187,8 +187,9 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
  * caching allocator at start-up, or a service held to a fixed, pre-reserved
  * budget -- because the workspace that oc_gptq_quantize grows with cudaMalloc
  * (and the device-wide synchronisation of the cudaFree before a regrowth)
- * would fail or stall there.  This entry point computes exactly what
- * oc_gptq_quantize computes, with the same arguments, but takes every byte of
+ * would fail or stall there.  This entry point takes the same steps as
+ * oc_gptq_quantize, with the same arguments (its trailing updates run on the
+ * CUDA cores in fp32, so results agree within rounding), but takes every byte of
  * scratch from one array built into the library (6 MiB per GPU, held by every
  * GPU that loads the library until the process exits) and never calls
  * cudaMalloc, cudaFree or any other allocating routine.  The caller still

@@ -1,0 +1,371 @@
+// fp32-accurate GEMM on the 5th-generation tensor cores (3xTF32):
+//   C  = alpha * A op(B)        (store)        or
+//   C += alpha * A op(B)        (accumulate: TMA reduce-add)
+// with A [M x K] and B [N x K] both row-major (op(B) = B^T), i.e. both operands
+// K-major in shared memory.  A product whose B is stored [K x N] passes the
+// transposed split copy instead (split_tf32 with transpose writes it).
+//
+// Every operand x is split once, outside this kernel, into x_hi = tf32(x) and
+// x_lo = tf32(x - x_hi); the product is accumulated as
+//   a_hi b_hi + a_hi b_lo + a_lo b_hi
+// in fp32 TMEM (the dropped a_lo b_lo term is ~2^-22 of a b).  The tensor
+// cores read both halves exactly, so the result carries about 21 bits.
+//
+// One persistent CTA per SM, 256 threads: warp 0 issues TMA loads (4 boxes of
+// 16 KB per 32-deep k slice: A_hi, A_lo, B_hi, B_lo, 128-byte swizzle,
+// 3-stage ring), warp 1 owns TMEM (two 128x128 fp32 accumulators) and issues
+// tcgen05.mma kind::tf32 M128 N128 K8 (12 per slice), warps 4..7 drain the
+// accumulator through swizzled 32x32 shared-memory boxes into TMA stores or
+// reduce-adds.  Triangular operands clip the k range of each tile.
+#include <algorithm>
+
+#include "oc_internal.cuh"
+#include "ptx_sm100.cuh"
+
+namespace oc {
+namespace {
+
+constexpr int BM = 128, BN = 128, BK = 32;  // BK fp32 = 128 bytes = one swizzle row
+constexpr int STAGES = 3;
+constexpr int TILE_BYTES = BM * BK * 4;      // 16 KB (A or B, one half)
+constexpr int STAGE_BYTES = 4 * TILE_BYTES;  // A_hi, A_lo, B_hi, B_lo
+constexpr int EPI_WARPS = 4;
+constexpr int EPI_BOX_BYTES = 32 * 32 * 4;
+constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BOX_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 1024;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr int THREADS = 256;
+
+struct Params {
+  int M, N, K;
+  int tiles_m, tiles_n;
+  unsigned flags;
+  float alpha;
+  int accumulate;
+  int* status;
+};
+
+__device__ __forceinline__ void k_range(const Params& p, int i0, int j0, int& kb, int& ke) {
+  kb = 0;
+  ke = p.K;
+  if (p.flags & kAUpper) kb = max(kb, i0);
+  if (p.flags & kALower) ke = min(ke, i0 + BM);
+  if (p.flags & kBLower) kb = max(kb, j0);
+  if (p.flags & kBUpper) ke = min(ke, j0 + BN);
+  kb = (kb / BK) * BK;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constant__ CUtensorMap mAl,
+                   const __grid_constant__ CUtensorMap mBh, const __grid_constant__ CUtensorMap mBl,
+                   const __grid_constant__ CUtensorMap mC, const Params p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* stage_base = smem;
+  unsigned char* epi_base = smem + STAGES * STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_base + EPI_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_tiles = p.tiles_m * p.tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&mAh);
+    prefetch_tensormap(&mAl);
+    prefetch_tensormap(&mBh);
+    prefetch_tensormap(&mBl);
+    prefetch_tensormap(&mC);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    uint64_t issued = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      const int i0 = (t % p.tiles_m) * BM, j0 = (t / p.tiles_m) * BN;
+      int kb, ke;
+      k_range(p, i0, j0, kb, ke);
+      for (int k0 = kb; k0 < ke; k0 += BK) {
+        const int s = static_cast<int>(issued % STAGES);
+        const uint32_t ph = static_cast<uint32_t>((issued / STAGES) & 1);
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&empty[s], ph ^ 1) && !*abort_flag;
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) { ok = false; break; }
+        if (lane == 0) {
+          unsigned char* st = stage_base + s * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          tma_load_2d(&mAh, &full[s], st, k0, i0);
+          tma_load_2d(&mAl, &full[s], st + TILE_BYTES, k0, i0);
+          tma_load_2d(&mBh, &full[s], st + 2 * TILE_BYTES, k0, j0);
+          tma_load_2d(&mBl, &full[s], st + 3 * TILE_BYTES, k0, j0);
+        }
+        __syncwarp();
+        ++issued;
+      }
+    }
+    if (lane == 0) {
+      if (!ok) {
+        record_error(p.status, kDevTimeout);
+        *abort_flag = 1;
+      }
+      const uint64_t first = issued > STAGES ? issued - STAGES : 0;
+      for (uint64_t q = first; q < issued; ++q) {
+        if (!mbar_wait(&full[q % STAGES], static_cast<uint32_t>((q / STAGES) & 1))) {
+          record_error(p.status, kDevTimeout);
+          break;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = instr_desc(2, 2, false, false, BM, BN);
+    uint64_t consumed = 0;
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
+      const int i0 = (t % p.tiles_m) * BM, j0 = (t / p.tiles_m) * BN;
+      int kb, ke;
+      k_range(p, i0, j0, kb, ke);
+      const int acc = it & 1;
+      int w = 1;
+      if (lane == 0) w = mbar_wait(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1));
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (!w) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t dcol = tmem_base + static_cast<uint32_t>(acc * BN);
+      for (int k0 = kb; k0 < ke; k0 += BK) {
+        const int s = static_cast<int>(consumed % STAGES);
+        const uint32_t ph = static_cast<uint32_t>((consumed / STAGES) & 1);
+        w = 1;
+        if (lane == 0) w = mbar_wait(&full[s], ph) && !*abort_flag;
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t sa = smem_u32(stage_base + s * STAGE_BYTES);
+          const uint32_t sah = sa, sal = sa + TILE_BYTES, sbh = sa + 2 * TILE_BYTES, sbl = sa + 3 * TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 8; ++kk) {
+            const uint64_t ah = smem_desc_sw128(sah + kk * 32, 16, 1024);
+            const uint64_t al = smem_desc_sw128(sal + kk * 32, 16, 1024);
+            const uint64_t bh = smem_desc_sw128(sbh + kk * 32, 16, 1024);
+            const uint64_t bl = smem_desc_sw128(sbl + kk * 32, 16, 1024);
+            const uint32_t first = (k0 == kb && kk == 0) ? 0u : 1u;
+            mma_tf32_ss(dcol, al, bh, idesc, first);
+            mma_tf32_ss(dcol, ah, bl, idesc, 1u);
+            mma_tf32_ss(dcol, ah, bh, idesc, 1u);
+          }
+          mma_commit(&empty[s]);
+        }
+        __syncwarp();
+        ++consumed;
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(&tfull[acc]);
+      __syncwarp();
+    }
+    if (lane == 0) {
+      if (!ok) {
+        record_error(p.status, kDevTimeout);
+        *abort_flag = 1;
+      }
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0)) record_error(p.status, kDevTimeout);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp - 4;
+    unsigned char* stage_buf = epi_base + q * 2 * EPI_BOX_BYTES;
+    int it = 0, nbuf = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+      const int i0 = (t % p.tiles_m) * BM, j0 = (t / p.tiles_m) * BN;
+      int kb, ke;
+      k_range(p, i0, j0, kb, ke);
+      const bool empty_k = kb >= ke;
+      const int acc = it & 1;
+      int w = 1;
+      if (lane == 0) w = mbar_wait(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1)) && !*abort_flag;
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (!w) { ok = false; break; }
+      tc_fence_after();
+      if (!(empty_k && p.accumulate)) {
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          if (!empty_k) {
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                   static_cast<uint32_t>(acc * BN + c * 32);
+            tmem_ld_32x32b_x32(taddr, r);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0u;
+          }
+          unsigned char* buf = stage_buf + (nbuf & 1) * EPI_BOX_BYTES;
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            float4 v;
+            v.x = __uint_as_float(r[4 * k + 0]) * p.alpha;
+            v.y = __uint_as_float(r[4 * k + 1]) * p.alpha;
+            v.z = __uint_as_float(r[4 * k + 2]) * p.alpha;
+            v.w = __uint_as_float(r[4 * k + 3]) * p.alpha;
+            *reinterpret_cast<float4*>(buf + lane * 128 + ((k ^ (lane & 7)) << 4)) = v;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (p.accumulate) tma_reduce_add_2d(&mC, buf, j0 + c * 32, i0 + 32 * q);
+            else tma_store_2d(&mC, buf, j0 + c * 32, i0 + 32 * q);
+            bulk_commit_group();
+          }
+          ++nbuf;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+    if (!ok && lane == 0) {
+      record_error(p.status, kDevTimeout);
+      *abort_flag = 1;
+    }
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// x_hi = tf32(x), x_lo = tf32(x - x_hi), both rounded to nearest (ties away).
+__device__ __forceinline__ float to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+__global__ void split_tf32_kernel(const float* __restrict__ src, int64_t rows, int64_t cols, int64_t lds,
+                                  float* __restrict__ hi, float* __restrict__ lo, int64_t ldd) {
+  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
+    for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < cols;
+         c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      const float x = src[r * lds + c];
+      const float h = to_tf32(x);
+      hi[r * ldd + c] = h;
+      lo[r * ldd + c] = to_tf32(x - h);
+    }
+  }
+}
+
+// Transposing split: hi[c][r], lo[c][r] from src[r][c], through 32x32 tiles.
+__global__ void split_tf32_t_kernel(const float* __restrict__ src, int64_t rows, int64_t cols, int64_t lds,
+                                    float* __restrict__ hi, float* __restrict__ lo, int64_t ldd) {
+  __shared__ float t[32][33];
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 32, c0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  for (int k = ty; k < 32; k += 8) {
+    const int64_t r = r0 + k, c = c0 + tx;
+    t[k][tx] = (r < rows && c < cols) ? src[r * lds + c] : 0.f;
+  }
+  __syncthreads();
+  for (int k = ty; k < 32; k += 8) {
+    const int64_t c = c0 + k, r = r0 + tx;  // output row c, column r
+    if (c < cols && r < rows) {
+      const float x = t[tx][k];
+      const float h = to_tf32(x);
+      hi[c * ldd + r] = h;
+      lo[c * ldd + r] = to_tf32(x - h);
+    }
+  }
+}
+
+void set_attr_once(int device) {
+  static bool done[64] = {false};
+  if (!done[device & 63]) {
+    check_cuda(cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
+               "cudaFuncSetAttribute(gemm_tf32x3)");
+    done[device & 63] = true;
+  }
+}
+
+}  // namespace
+
+void split_tf32(const Ctx& c, const float* src, int64_t rows, int64_t cols, int64_t lds, float* hi, float* lo,
+                int64_t ldd, bool transpose) {
+  if (rows <= 0 || cols <= 0) return;
+  if (transpose) {
+    if ((rows + 31) / 32 > 65535) fail(OC_ERR_INVALID_ARG, "split_tf32: too many rows");
+    dim3 grid(static_cast<unsigned>((cols + 31) / 32), static_cast<unsigned>((rows + 31) / 32));
+    split_tf32_t_kernel<<<grid, dim3(32, 8), 0, c.stream>>>(src, rows, cols, lds, hi, lo, ldd);
+    check_launch("split_tf32_t_kernel");
+    return;
+  }
+  dim3 grid(static_cast<unsigned>(std::min<int64_t>((cols + 255) / 256, 64)),
+            static_cast<unsigned>(std::min<int64_t>(rows, 8192)));
+  split_tf32_kernel<<<grid, 256, 0, c.stream>>>(src, rows, cols, lds, hi, lo, ldd);
+  check_launch("split_tf32_kernel");
+}
+
+void gemm_tf32x3(const Ctx& c, int64_t M, int64_t N, int64_t K, float alpha, const float* A_hi,
+                 const float* A_lo, int64_t lda, const float* B_hi, const float* B_lo, int64_t ldb,
+                 bool accumulate, float* C, int64_t ldc, unsigned flags) {
+  if (M <= 0 || N <= 0) return;
+  if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || K > (int64_t(1) << 30))
+    fail(OC_ERR_INVALID_ARG, "gemm_tf32x3: size too large");
+  const CUtensorMap mAh = make_tmap_2d(A_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, M, K, lda, BM, BK, Swz::B128);
+  const CUtensorMap mAl = make_tmap_2d(A_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, M, K, lda, BM, BK, Swz::B128);
+  const CUtensorMap mBh = make_tmap_2d(B_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, K, ldb, BN, BK, Swz::B128);
+  const CUtensorMap mBl = make_tmap_2d(B_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, K, ldb, BN, BK, Swz::B128);
+  const CUtensorMap mC = make_tmap_2d(C, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, M, N, ldc, 32, 32, Swz::B128);
+  Params p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.tiles_m = static_cast<int>((M + BM - 1) / BM);
+  p.tiles_n = static_cast<int>((N + BN - 1) / BN);
+  p.flags = flags;
+  p.alpha = alpha;
+  p.accumulate = accumulate ? 1 : 0;
+  p.status = c.status;
+  const int64_t n_tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+  const int grid = static_cast<int>(std::min<int64_t>(n_tiles, c.sm_count));
+  set_attr_once(c.device);
+  gemm_tf32x3_kernel<<<grid, THREADS, SMEM_BYTES, c.stream>>>(mAh, mAl, mBh, mBl, mC, p);
+  check_launch("gemm_tf32x3_kernel");
+}
+
+}  // namespace oc

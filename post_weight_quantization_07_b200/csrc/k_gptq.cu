@@ -16,7 +16,7 @@ namespace oc {
 namespace {
 
 constexpr int SB = 128;          // sweep block width
-constexpr int SWEEP_WARPS = 8;
+constexpr int SWEEP_WARPS = 16;
 
 __device__ __forceinline__ void grid_from_minmax(float xmin, float xmax, float maxq, float& s,
                                                  float& z) {
@@ -82,6 +82,11 @@ sweep_block_kernel(float* __restrict__ Wp, int64_t m, int64_t n, const float* __
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ng = n / G;
   const int64_t col0 = j1 + 4 * lane;  // first column of this lane
+  // Group starts inside this block (all 32-bit, no division in the loop): a
+  // group of at most one block (G divides 128) starts wherever j % G == 0; a
+  // wider group can only start at the block's first column.
+  const bool g_small = G <= SB;
+  const bool block_starts_group = (j1 % G) == 0;
   for (int64_t r = static_cast<int64_t>(blockIdx.x) * SWEEP_WARPS + warp; r < m;
        r += static_cast<int64_t>(gridDim.x) * SWEEP_WARPS) {
     float* wrow = Wp + r * n;
@@ -89,19 +94,18 @@ sweep_block_kernel(float* __restrict__ Wp, int64_t m, int64_t n, const float* __
     unsigned qv[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const int64_t col = col0 + c;
-      w[c] = (4 * lane + c < bw) ? wrow[col] : 0.f;
+      w[c] = (4 * lane + c < bw) ? wrow[col0 + c] : 0.f;
       s[c] = 1.f;
       z[c] = 0.f;
       ev[c] = 0.f;
       qv[c] = 0u;
       if (static_groups && 4 * lane + c < bw) {
-        const int64_t g = perm[col] / G;
+        const int g = perm[col0 + c] / G;
         s[c] = scales[r * ng + g];
         z[c] = zeros[r * ng + g];
       }
     }
-    if (!static_groups && (j1 % G) != 0) {
+    if (!static_groups && !block_starts_group) {
       // a group wider than the block started in an earlier block: its grid
       // was written by that block's sweep
       const int64_t g = j1 / G;
@@ -113,11 +117,10 @@ sweep_block_kernel(float* __restrict__ Wp, int64_t m, int64_t n, const float* __
       }
     }
     for (int j = 0; j < bw; ++j) {
-      const int64_t gj = j1 + j;
-      if (!static_groups && (gj % G) == 0) {
-        // group [gj, gj + G): min/max of its current values
+      if (!static_groups && (g_small ? ((j & (G - 1)) == 0) : (j == 0 && block_starts_group))) {
+        // group [j1 + j, j1 + j + G): min/max of its current values
         float xmin = INFINITY, xmax = -INFINITY;
-        if (G <= SB) {
+        if (g_small) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const int k = 4 * lane + c;
@@ -130,7 +133,7 @@ sweep_block_kernel(float* __restrict__ Wp, int64_t m, int64_t n, const float* __
           // the group starts at this block and extends beyond it; every column
           // of it is current (earlier blocks' updates are applied, this block's
           // have not started)
-          for (int64_t k = gj + lane; k < gj + G; k += 32) {
+          for (int64_t k = j1 + lane; k < j1 + G; k += 32) {
             const float v = wrow[k];
             xmin = fminf(xmin, v);
             xmax = fmaxf(xmax, v);
@@ -142,20 +145,22 @@ sweep_block_kernel(float* __restrict__ Wp, int64_t m, int64_t n, const float* __
         }
         float gs, gz;
         grid_from_minmax(xmin, xmax, maxq, gs, gz);
-        const int64_t g = gj / G;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          if ((col0 + c) / G == g) {
+          const int k = 4 * lane + c;
+          if (!g_small || (k >= j && k < j + G)) {
             s[c] = gs;
             z[c] = gz;
           }
         }
         if (lane == 0) {
+          const int64_t g = (j1 + j) / G;
           scales[r * ng + g] = gs;
           zeros[r * ng + g] = gz;
         }
       }
       const int owner = j >> 2, comp = j & 3;
+      const float4 u = *reinterpret_cast<const float4*>(&Ub[j * SB + 4 * lane]);
       float e = 0.f;
       if (lane == owner) {
         float wj = w[0], sj = s[0], zj = z[0];
@@ -177,7 +182,6 @@ sweep_block_kernel(float* __restrict__ Wp, int64_t m, int64_t n, const float* __
           }
       }
       e = __shfl_sync(0xffffffffu, e, owner);
-      const float4 u = *reinterpret_cast<const float4*>(&Ub[j * SB + 4 * lane]);
       w[0] = fmaf(-e, u.x, w[0]);
       w[1] = fmaf(-e, u.y, w[1]);
       w[2] = fmaf(-e, u.z, w[2]);
@@ -275,6 +279,8 @@ void launch_sweep_block(const Ctx& c, float* Wp, int64_t m, int64_t n, const flo
   const int64_t rows_per_cta = SWEEP_WARPS;
   const int64_t want = (m + rows_per_cta - 1) / rows_per_cta;
   const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(c.sm_count) * 3));
+  // (16 warps and 64 KB of shared memory per CTA: three CTAs per SM, so 4096
+  // rows run in a single wave)
   sweep_block_kernel<<<grid, SWEEP_WARPS * 32, smem, c.stream>>>(
       Wp, m, n, U, j1, G, static_cast<float>((1 << wbits) - 1), static_groups ? 1 : 0, perm, scales, zeros,
       codes8, Err);

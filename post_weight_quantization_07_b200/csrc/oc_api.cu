@@ -281,20 +281,26 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
       return finish(c);
     }
     Carve sizing{nullptr};
-    sizing.take<float>(nn);                       // D -> M -> U
+    sizing.take<float>(nn);                       // d -> M -> U
     if (!H_opt) sizing.take<float>(nn);           // Hs
-    sizing.take<float>(nn);                       // X (inverse factor of the reversed matrix)
-    sizing.take<float>(nn / 2 + 4096);            // recursion scratch
-    sizing.take<float>(mn);                       // G
-    sizing.take<float>(mn);                       // T
+    sizing.take<float>(nn);                       // d_hi -> inverse factor -> U_hi
+    sizing.take<float>(nn + 4096);                // d_lo -> recursion scratch -> U_lo
+    sizing.take<float>(nn);                       // (U^T)_hi
+    sizing.take<float>(nn);                       // (U^T)_lo
+    sizing.take<float>(mn);                       // W_hi -> G_hi -> T_hi
+    sizing.take<float>(mn);                       // W_lo -> G_lo -> T_lo
+    sizing.take<float>(mn);                       // G -> T
     sizing.take<DiagStats>(1);
     Carve cv{workspace(c, sizing.off + 256)};
     float* D = cv.take<float>(nn);
     float* Hs = H_opt ? nullptr : cv.take<float>(nn);
     float* Xi = cv.take<float>(nn);
-    float* scratch = cv.take<float>(nn / 2 + 4096);
+    float* scratch = cv.take<float>(nn + 4096);
+    float* UTh = cv.take<float>(nn);
+    float* UTl = cv.take<float>(nn);
+    float* Ph = cv.take<float>(mn);
+    float* Pl = cv.take<float>(mn);
     float* G = cv.take<float>(mn);
-    float* T = cv.take<float>(mn);
     DiagStats* stats = cv.take<DiagStats>(1);
 
     // d = X^T Xhat - Xhat^T Xhat  (the second term from H = 2 Xhat^T Xhat)
@@ -313,9 +319,11 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
       launch_sub_half(c, D, Hp, n);
     }
     {
-      // G = W d
+      // G = W d on the tensor cores (3xTF32 from split operands)
       PhaseScope ps(c, kPhQepWDelta);
-      gemm_f32(c, false, false, m, n, n, 1.f, W, n, D, n, 0.f, G, n, kANone);
+      split_tf32(c, D, n, n, n, Xi, scratch, n, true);  // d^T: B operands are stored [N x K]
+      split_tf32(c, W, m, n, n, Ph, Pl, n);
+      gemm_tf32x3(c, m, n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, G, n, kANone);
     }
     {
       // 2A = Hp + damp mean(diag Hp) I = R R^T;  U = R^-1 upper, A^-1 = 2 U^T U
@@ -328,9 +336,18 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
       // W_out = W + alpha G A^-1 = W + 2 alpha (G U^T) U
       PhaseScope ps(c, kPhQepApply);
       const float* U = D;
-      gemm_f32(c, false, true, m, n, n, 1.f, G, n, U, n, 0.f, T, n, kBLower);
+      float* Uh = Xi;
+      float* Ul = scratch;
+      split_tf32(c, U, n, n, n, Uh, Ul, n);
+      split_tf32(c, U, n, n, n, UTh, UTl, n, true);
+      split_tf32(c, G, m, n, n, Ph, Pl, n);
+      float* T = G;
+      // T = G U^T (B stored = U; op(B) = U^T is lower triangular)
+      gemm_tf32x3(c, m, n, n, 1.f, Ph, Pl, n, Uh, Ul, n, false, T, n, kBLower);
+      split_tf32(c, T, m, n, n, Ph, Pl, n);
       if (W_out != W) launch_copy_f32(c, W, W_out, static_cast<int64_t>(mn));
-      gemm_f32(c, false, false, m, n, n, 2.f * alpha, T, n, U, n, 1.f, W_out, n, kBUpper);
+      // W_out += 2 alpha T U (B stored = U^T; op(B) = U is upper triangular)
+      gemm_tf32x3(c, m, n, n, 2.f * alpha, Ph, Pl, n, UTh, UTl, n, true, W_out, n, kBUpper);
     }
     return finish(c);
   });
@@ -357,21 +374,25 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
     const size_t nn = static_cast<size_t>(n) * n, mn = static_cast<size_t>(m) * n;
     Carve sizing{nullptr};
     sizing.take<float>(nn);            // M -> U
-    sizing.take<float>(nn);            // X
-    sizing.take<float>(nn / 2 + 4096); // scratch
+    sizing.take<float>(nn);            // inverse factor -> U_hi
+    sizing.take<float>(nn + 4096);     // recursion scratch -> U_lo
     sizing.take<float>(mn);            // Wp
     sizing.take<unsigned char>(mn);    // codes8
     sizing.take<float>(static_cast<size_t>(m) * 128);  // Err
+    sizing.take<float>(static_cast<size_t>(m) * 128);  // Err_hi
+    sizing.take<float>(static_cast<size_t>(m) * 128);  // Err_lo
     sizing.take<int32_t>(2 * static_cast<size_t>(n));  // perm | inverse
     sizing.take<unsigned char>(n);     // dead
     sizing.take<DiagStats>(1);
     Carve cv{workspace(c, sizing.off + 256)};
     float* M = cv.take<float>(nn);
     float* Xi = cv.take<float>(nn);
-    float* scratch = cv.take<float>(nn / 2 + 4096);
+    float* scratch = cv.take<float>(nn + 4096);
     float* Wp = cv.take<float>(mn);
     unsigned char* codes8 = cv.take<unsigned char>(mn);
     float* Err = cv.take<float>(static_cast<size_t>(m) * 128);
+    float* Errh = cv.take<float>(static_cast<size_t>(m) * 128);
+    float* Errl = cv.take<float>(static_cast<size_t>(m) * 128);
     int32_t* perm = cv.take<int32_t>(2 * static_cast<size_t>(n));
     unsigned char* dead = cv.take<unsigned char>(n);
     DiagStats* stats = cv.take<DiagStats>(1);
@@ -385,8 +406,11 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
       factor_inverse_upper(c, M, Xi, scratch, M, n);
     }
     const float* U = M;
+    float* UTh = Xi;
+    float* UTl = scratch;
     {
       PhaseScope ps(c, kPhGptqPrep);
+      split_tf32(c, U, n, n, n, UTh, UTl, n, true);
       launch_permute_w(c, W, m, n, perm, dead, Wp);
       if (act_order) launch_static_grid(c, W, m, n, static_cast<int>(G), wbits, dead, scales, zeros);
     }
@@ -399,8 +423,12 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
                            codes8, Err);
       }
       if (j2 < n) {
+        // W[:, j2:] -= Err U[j1:j2, j2:] on the tensor cores (3xTF32)
         PhaseScope ps(c, kPhGptqTrailing);
-        gemm_f32(c, false, false, m, n - j2, bw, -1.f, Err, 128, U + j1 * n + j2, n, 1.f, Wp + j2, n, kANone);
+        split_tf32(c, Err, m, bw, 128, Errh, Errl, 128);
+        // B stored = U^T[j2:, j1:j2] (rows j2.., columns j1..j1+bw of the transpose)
+        gemm_tf32x3(c, m, n - j2, bw, -1.f, Errh, Errl, 128, UTh + j2 * n + j1, UTl + j2 * n + j1, n, true,
+                    Wp + j2, n, kANone);
       }
     }
     {

@@ -114,6 +114,20 @@ void gemm_f32(const Ctx& c, bool tA, bool tB, int64_t M, int64_t N, int64_t K, f
               const float* A, int64_t lda, const float* B, int64_t ldb, float beta, float* C,
               int64_t ldc, unsigned flags);
 
+// x_hi = tf32(x), x_lo = tf32(x - x_hi) of a rows x cols block of src
+// (leading dimension lds); written untransposed (ldd) or, with transpose,
+// as the cols x rows transpose (ldd = leading dimension of the transpose).
+void split_tf32(const Ctx& c, const float* src, int64_t rows, int64_t cols, int64_t lds, float* hi,
+                float* lo, int64_t ldd, bool transpose = false);
+
+// fp32-accurate tensor-core GEMM from split operands: C (+)= alpha A B^T with
+// A [M x K] (lda) and B [N x K] (ldb) row-major; accumulate selects C += over
+// C =.  Flags describe the triangles of A and of op(B) = B^T.  Pointers and
+// leading dimensions must allow 16-byte aligned TMA rows.
+void gemm_tf32x3(const Ctx& c, int64_t M, int64_t N, int64_t K, float alpha, const float* A_hi,
+                 const float* A_lo, int64_t lda, const float* B_hi, const float* B_lo, int64_t ldb,
+                 bool accumulate, float* C, int64_t ldc, unsigned flags);
+
 // U = upper Cholesky factor of (H_prepared)^-1, where H_prepared is formed by
 // `launch_build_reversed` into M (consumed).  Scratch must hold n*n/2 + 4096
 // floats.  X receives L^-1 of the reversed matrix (lower), U its reversal.

@@ -5,8 +5,9 @@
 // a service that runs under a fixed, pre-reserved memory budget, or any host
 // code where a cudaMalloc (and the device-wide synchronisation a cudaFree
 // brings) at an arbitrary point is not acceptable.  oc_gptq_quantize_noalloc
-// serves them: it runs exactly the kernels of oc_gptq_quantize, but takes all
-// of its scratch memory from one fixed array that is part of the library image
+// serves them: it takes the same steps as oc_gptq_quantize (its trailing
+// updates run on the CUDA cores in fp32, which needs no split copies of the
+// factor), but takes all of its scratch memory from one fixed array that is part of the library image
 // (g_noalloc_scratch below), so it never calls cudaMalloc, cudaFree or any
 // other allocating routine.  The price is a size limit (kNoallocBytes of
 // scratch, enough for d_in = 512 with up to 1024 output rows) and the memory
