@@ -14,16 +14,17 @@
 //                Y = L21 X11                               (GEMM, before the next recursion)
 //                L22 = chol(A22'), X22 = L22^-1            (recurse)
 //                X21 = -X22 Y                              (GEMM)
-// with 64x64 leaves factored and inverted inside one CTA.
+// with 128x128 leaves factored and inverted inside one CTA.
 #include <algorithm>
 #include <cmath>
+#include <vector>
 
 #include "oc_internal.cuh"
 
 namespace oc {
 namespace {
 
-constexpr int LEAF = 64;
+constexpr int LEAF = 128;
 
 // ---------------------------------------------------------------- diag stats
 // One block: dead mask, non-finite check and the dampening constant
@@ -135,65 +136,202 @@ __global__ void build_reversed_kernel(const float* __restrict__ H, int64_t n,
 }
 
 // ---------------------------------------------------------------- leaf
-// Cholesky of the s x s diagonal block at M (lower part read) and the inverse
-// of its factor, written to X (lower, explicit zeros above the diagonal).
-// Right-looking elimination without normalising the pivot column:
-//   A[i][j] -= A[i][k] A[j][k] / A[k][k]   for k < j <= i,
-// so that afterwards L[i][k] = A[i][k] / sqrt(A[k][k]); one barrier per column.
+// Cholesky of an s x s (s <= 128) diagonal block at M (lower part read) and
+// the inverse of its factor, written to X (lower, explicit zeros above), in
+// one CTA with the whole block in shared memory.  The block is split
+// recursively, 128 -> 64 -> 32, with the same four products as the outer
+// recursion:
+//   X11 = L11^-1 (recurse);  T = A21 X11^T (= L21);  A22 -= T T^T;
+//   Y = T X11;  X22 = L22^-1 (recurse);  X21 = -X22 Y.
+// A 32x32 block is factored and inverted by one warp: lane i holds row i in
+// registers; column k of L reaches the other lanes by shuffles; the inverse is
+// forward substitution per column (lane j owns column j of X) reading L from
+// shared memory.  Rows and columns beyond s are padded with the identity.
+constexpr int LDA = LEAF + 1;      // padded leading dimensions (bank spread)
+constexpr int LDT = LEAF / 2 + 1;
+
+struct LeafSmem {
+  float A[LEAF * LDA];
+  float X[LEAF * LDA];
+  float T[(LEAF / 2) * LDT];       // L21 of the 128 level; temporaries of the 64 level
+  float Y[(LEAF / 2) * LDT];       // Y of the 128 level (lives across the right half)
+  float L32[32 * 33];              // factor of the current 32 block
+};
+
+__device__ __forceinline__ void warp_chol_inv32(LeafSmem& sm, int off, int* status) {
+  const int lane = threadIdx.x & 31;
+  float a[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) a[j] = (j <= lane) ? sm.A[(off + lane) * LDA + off + j] : 0.f;
+  bool bad = false;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const float d = __shfl_sync(0xffffffffu, a[k], k);
+    if (!(d > 0.f) || !isfinite(d)) bad = true;
+    const float rsd = rsqrtf(d);
+    const float lk = a[k] * rsd;  // L[lane][k] (0 above the diagonal)
+    a[k] = lk;
+#pragma unroll
+    for (int j = k + 1; j < 32; ++j) {
+      const float ljk = __shfl_sync(0xffffffffu, lk, j);
+      if (lane >= j) a[j] = fmaf(-lk, ljk, a[j]);
+    }
+  }
+  if (bad && lane == 0) record_error(status, kDevNotSpd);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) sm.L32[lane * 33 + j] = a[j];
+  __syncwarp();
+  // column `lane` of X = L^-1: x_i = (delta_i,lane - sum_{k<i} L_ik x_k) / L_ii
+  float x[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    float acc = (i == lane) ? 1.f : 0.f;
+#pragma unroll
+    for (int k = 0; k < i; ++k) acc = fmaf(-sm.L32[i * 33 + k], x[k], acc);
+    x[i] = acc / sm.L32[i * 33 + i];
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) sm.X[(off + i) * LDA + off + lane] = x[i];
+}
+
+// The four products of one recursion node of half width H inside the CTA
+// (256 threads, each a TR x TC register tile of the H x H outputs).
+template <int H>
+__device__ __forceinline__ void node_pre(LeafSmem& sm, int off, float* T, int ldt, float* Y, int ldy) {
+  constexpr int TR = (H == 64) ? 4 : 2, TC = TR;
+  constexpr int NTC = H / TC;
+  const int t = threadIdx.x;
+  const int i0 = (t / NTC) * TR, j0 = (t % NTC) * TC;
+  const float* A21 = &sm.A[(off + H) * LDA + off];
+  float* A22 = &sm.A[(off + H) * LDA + off + H];
+  const float* X11 = &sm.X[off * LDA + off];
+  // T = A21 X11^T: T[i][j] = sum_{k <= j} A21[i][k] X11[j][k]
+  {
+    float acc[TR][TC] = {};
+    for (int k = 0; k < j0 + TC; ++k) {
+      float av[TR], bv[TC];
+#pragma unroll
+      for (int r = 0; r < TR; ++r) av[r] = A21[(i0 + r) * LDA + k];
+#pragma unroll
+      for (int c = 0; c < TC; ++c) bv[c] = X11[(j0 + c) * LDA + k];
+#pragma unroll
+      for (int r = 0; r < TR; ++r)
+#pragma unroll
+        for (int c = 0; c < TC; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+    }
+#pragma unroll
+    for (int r = 0; r < TR; ++r)
+#pragma unroll
+      for (int c = 0; c < TC; ++c) T[(i0 + r) * ldt + j0 + c] = acc[r][c];
+  }
+  __syncthreads();
+  // A22 -= T T^T (tiles touching the lower triangle)
+  if (j0 <= i0 + TR - 1) {
+    float acc[TR][TC] = {};
+    for (int k = 0; k < H; ++k) {
+      float av[TR], bv[TC];
+#pragma unroll
+      for (int r = 0; r < TR; ++r) av[r] = T[(i0 + r) * ldt + k];
+#pragma unroll
+      for (int c = 0; c < TC; ++c) bv[c] = T[(j0 + c) * ldt + k];
+#pragma unroll
+      for (int r = 0; r < TR; ++r)
+#pragma unroll
+        for (int c = 0; c < TC; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+    }
+#pragma unroll
+    for (int r = 0; r < TR; ++r)
+#pragma unroll
+      for (int c = 0; c < TC; ++c) A22[(i0 + r) * LDA + j0 + c] -= acc[r][c];
+  }
+  // Y = T X11: Y[i][j] = sum_{k >= j} T[i][k] X11[k][j]
+  {
+    float acc[TR][TC] = {};
+    for (int k = j0; k < H; ++k) {
+      float av[TR], bv[TC];
+#pragma unroll
+      for (int r = 0; r < TR; ++r) av[r] = T[(i0 + r) * ldt + k];
+#pragma unroll
+      for (int c = 0; c < TC; ++c) bv[c] = X11[k * LDA + j0 + c];
+#pragma unroll
+      for (int r = 0; r < TR; ++r)
+#pragma unroll
+        for (int c = 0; c < TC; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+    }
+#pragma unroll
+    for (int r = 0; r < TR; ++r)
+#pragma unroll
+      for (int c = 0; c < TC; ++c) Y[(i0 + r) * ldy + j0 + c] = acc[r][c];
+  }
+  __syncthreads();
+}
+
+template <int H>
+__device__ __forceinline__ void node_post(LeafSmem& sm, int off, const float* Y, int ldy) {
+  constexpr int TR = (H == 64) ? 4 : 2, TC = TR;
+  constexpr int NTC = H / TC;
+  const int t = threadIdx.x;
+  const int i0 = (t / NTC) * TR, j0 = (t % NTC) * TC;
+  const float* X22 = &sm.X[(off + H) * LDA + off + H];
+  float* X21 = &sm.X[(off + H) * LDA + off];
+  // X21 = -X22 Y: X21[i][j] = -sum_{k <= i} X22[i][k] Y[k][j]
+  float acc[TR][TC] = {};
+  for (int k = 0; k < i0 + TR; ++k) {
+    float av[TR], bv[TC];
+#pragma unroll
+    for (int r = 0; r < TR; ++r) av[r] = X22[(i0 + r) * LDA + k];
+#pragma unroll
+    for (int c = 0; c < TC; ++c) bv[c] = Y[k * ldy + j0 + c];
+#pragma unroll
+    for (int r = 0; r < TR; ++r)
+#pragma unroll
+      for (int c = 0; c < TC; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+  }
+#pragma unroll
+  for (int r = 0; r < TR; ++r)
+#pragma unroll
+    for (int c = 0; c < TC; ++c) X21[(i0 + r) * LDA + j0 + c] = -acc[r][c];
+  __syncthreads();
+}
+
+__device__ __forceinline__ void leaf32(LeafSmem& sm, int off, int* status) {
+  if ((threadIdx.x >> 5) == 0) warp_chol_inv32(sm, off, status);
+  __syncthreads();
+}
+
+// 64 block at `off`; its temporaries live in sm.T (T at 0, Y at 32 rows on).
+__device__ __forceinline__ void leaf64(LeafSmem& sm, int off, int* status) {
+  float* T = sm.T;
+  float* Y = sm.T + 32 * 33;
+  leaf32(sm, off, status);
+  node_pre<32>(sm, off, T, 33, Y, 33);
+  leaf32(sm, off + 32, status);
+  node_post<32>(sm, off, Y, 33);
+}
+
 __global__ void __launch_bounds__(256) leaf_chol_inv_kernel(const float* __restrict__ M, float* __restrict__ X,
                                                             int64_t ld, int s, int* status) {
-  __shared__ float A[LEAF][LEAF + 1];
-  __shared__ float B[LEAF][LEAF + 1];
+  extern __shared__ __align__(16) float leaf_smem[];
+  LeafSmem& sm = *reinterpret_cast<LeafSmem*>(leaf_smem);
   const int t = threadIdx.x;
   for (int e = t; e < LEAF * LEAF; e += blockDim.x) {
     const int i = e / LEAF, j = e % LEAF;
     float v = 0.f;
-    if (i < s && j <= i) v = M[static_cast<int64_t>(i) * ld + j];
-    else if (i == j) v = 1.f;  // padding rows beyond s: identity
-    A[i][j] = v;
-    B[i][j] = (i == j) ? 1.f : 0.f;
+    if (j <= i) {
+      if (i < s) v = M[static_cast<int64_t>(i) * ld + j];
+      else if (i == j) v = 1.f;
+    }
+    sm.A[i * LDA + j] = v;
+    sm.X[i * LDA + j] = 0.f;
   }
   __syncthreads();
-  for (int k = 0; k < LEAF - 1; ++k) {
-    const float inv_piv = 1.f / A[k][k];
-    for (int e = t; e < (LEAF - 1 - k) * (LEAF - 1 - k); e += blockDim.x) {
-      const int i = k + 1 + e / (LEAF - 1 - k);
-      const int j = k + 1 + e % (LEAF - 1 - k);
-      if (j <= i) A[i][j] -= A[i][k] * A[j][k] * inv_piv;
-    }
-    __syncthreads();
-  }
-  // pivots, then normalise: L[i][k] = A[i][k] / sqrt(A[k][k])
-  __shared__ float rs[LEAF];
-  if (t < LEAF) {
-    const float piv = A[t][t];
-    if (!(piv > 0.f) || !isfinite(piv)) {
-      record_error(status, kDevNotSpd);
-      rs[t] = 0.f;
-    } else {
-      rs[t] = rsqrtf(piv);
-    }
-  }
-  __syncthreads();
-  for (int e = t; e < LEAF * LEAF; e += blockDim.x) {
-    const int i = e / LEAF, k = e % LEAF;
-    A[i][k] = (k <= i) ? A[i][k] * rs[k] : 0.f;
-  }
-  __syncthreads();
-  // Forward substitution L Y = I for all columns: at step k, rows i > k take
-  // B[i][j] -= L[i][k] * B[k][j] / L[k][k] for j <= k; then X = B / diag(L).
-  for (int k = 0; k < LEAF - 1; ++k) {
-    const float inv_lkk = 1.f / A[k][k];
-    for (int e = t; e < (LEAF - 1 - k) * (k + 1); e += blockDim.x) {
-      const int i = k + 1 + e / (k + 1);
-      const int j = e % (k + 1);
-      B[i][j] -= A[i][k] * B[k][j] * inv_lkk;
-    }
-    __syncthreads();
-  }
+  leaf64(sm, 0, status);
+  node_pre<64>(sm, 0, sm.T, LDT, sm.Y, LDT);
+  leaf64(sm, 64, status);
+  node_post<64>(sm, 0, sm.Y, LDT);
   for (int e = t; e < s * s; e += blockDim.x) {
     const int i = e / s, j = e % s;
-    X[static_cast<int64_t>(i) * ld + j] = (j <= i) ? B[i][j] / A[i][i] : 0.f;
+    X[static_cast<int64_t>(i) * ld + j] = (j <= i) ? sm.X[i * LDA + j] : 0.f;
   }
 }
 
@@ -205,38 +343,104 @@ __global__ void reverse_kernel(const float* __restrict__ X, float* __restrict__ 
   U[e] = X[(n - 1 - i) * n + (n - 1 - j)];
 }
 
-void chol_inv_rec(const Ctx& c, float* M, float* X, int64_t ld, int64_t off, int64_t s,
-                  float* scratch) {
+// Nodes whose halves are at least this wide run their four products on the
+// tensor cores (3xTF32 from split copies); smaller ones are latency bound and
+// stay on the CUDA cores.
+constexpr int64_t kTensorNode = 512;
+
+// Split of a node of width s into halves h + r (h a multiple of the leaf).
+inline int64_t node_half(int64_t s) {
+  const int64_t nblk = (s + LEAF - 1) / LEAF;
+  return std::max<int64_t>(1, nblk / 2) * LEAF;
+}
+
+// Largest split-copy area any tensor-core node of the recursion needs.
+size_t split_need(int64_t s) {
+  if (s <= LEAF) return 0;
+  const int64_t h = node_half(s), r = s - h;
+  size_t here = 0;
+  if (h >= kTensorNode) {
+    const size_t before = 2 * static_cast<size_t>(r * h + h * h + h * h + r * h);
+    const size_t after = 2 * static_cast<size_t>(h * r + r * r);
+    here = std::max(before, after);
+  }
+  return std::max(here, std::max(split_need(h), split_need(r)));
+}
+
+void chol_inv_rec(const Ctx& c, float* M, float* X, int64_t ld, int64_t off, int64_t s, float* scratch,
+                  float* split) {
   float* Md = M + off * ld + off;
   float* Xd = X + off * ld + off;
   if (s <= LEAF) {
-    leaf_chol_inv_kernel<<<1, 256, 0, c.stream>>>(Md, Xd, ld, static_cast<int>(s), c.status);
+    static bool attr_done[64] = {false};
+    if (!attr_done[c.device & 63]) {
+      check_cuda(cudaFuncSetAttribute(leaf_chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(sizeof(LeafSmem))),
+                 "cudaFuncSetAttribute(leaf)");
+      attr_done[c.device & 63] = true;
+    }
+    leaf_chol_inv_kernel<<<1, 256, sizeof(LeafSmem), c.stream>>>(Md, Xd, ld, static_cast<int>(s), c.status);
     check_launch("leaf_chol_inv_kernel");
     return;
   }
-  const int64_t nblk = (s + LEAF - 1) / LEAF;
-  const int64_t h = std::max<int64_t>(1, nblk / 2) * LEAF;
+  const int64_t h = node_half(s);
   const int64_t r = s - h;
-  chol_inv_rec(c, M, X, ld, off, h, scratch);
+  chol_inv_rec(c, M, X, ld, off, h, scratch, split);
   float* Y = scratch;
   float* T = scratch + r * h;
   const float* M21 = M + (off + h) * ld + off;
   float* M22 = M + (off + h) * ld + (off + h);
   const float* X11 = Xd;
-  // L21 = A21 X11^T
-  gemm_f32(c, false, true, r, h, h, 1.f, M21, ld, X11, ld, 0.f, T, h, kBUpper);
-  // A22 -= L21 L21^T (lower tiles only)
-  gemm_f32(c, false, true, r, r, h, -1.f, T, h, T, h, 1.f, M22, ld, kCLowerOnly);
-  // Y = L21 X11
-  gemm_f32(c, false, false, r, h, h, 1.f, T, h, X11, ld, 0.f, Y, h, kBLower);
-  chol_inv_rec(c, M, X, ld, off + h, r, scratch + r * h);
-  // X21 = -X22 Y
   const float* X22 = X + (off + h) * ld + (off + h);
   float* X21 = X + (off + h) * ld + off;
-  gemm_f32(c, false, false, r, h, r, -1.f, X22, ld, Y, h, 0.f, X21, ld, kALower);
+  const bool tensor = split != nullptr && h >= kTensorNode;
+  if (tensor) {
+    // split copies (hi, lo) in `split`: [M21 | X11 | X11^T | T], then [Y^T | X22]
+    float* m21h = split;
+    float* m21l = m21h + r * h;
+    float* x11h = m21l + r * h;
+    float* x11l = x11h + h * h;
+    float* x11th = x11l + h * h;
+    float* x11tl = x11th + h * h;
+    float* th = x11tl + h * h;
+    float* tl = th + r * h;
+    split_tf32(c, M21, r, h, ld, m21h, m21l, h);
+    split_tf32(c, X11, h, h, ld, x11h, x11l, h);
+    split_tf32(c, X11, h, h, ld, x11th, x11tl, h, true);
+    // L21 = A21 X11^T  (B stored = X11, op(B) = X11^T upper)
+    gemm_tf32x3(c, r, h, h, 1.f, m21h, m21l, h, x11h, x11l, h, false, T, h, kBUpper);
+    split_tf32(c, T, r, h, h, th, tl, h);
+    // A22 -= L21 L21^T  (lower tiles)
+    gemm_tf32x3(c, r, r, h, -1.f, th, tl, h, th, tl, h, true, M22, ld, kCLowerOnly);
+    // Y = L21 X11  (B stored = X11^T, op(B) = X11 lower)
+    gemm_tf32x3(c, r, h, h, 1.f, th, tl, h, x11th, x11tl, h, false, Y, h, kBLower);
+  } else {
+    // L21 = A21 X11^T
+    gemm_f32(c, false, true, r, h, h, 1.f, M21, ld, X11, ld, 0.f, T, h, kBUpper);
+    // A22 -= L21 L21^T (lower tiles only)
+    gemm_f32(c, false, true, r, r, h, -1.f, T, h, T, h, 1.f, M22, ld, kCLowerOnly);
+    // Y = L21 X11
+    gemm_f32(c, false, false, r, h, h, 1.f, T, h, X11, ld, 0.f, Y, h, kBLower);
+  }
+  chol_inv_rec(c, M, X, ld, off + h, r, scratch + r * h, split);
+  if (tensor) {
+    float* yth = split;
+    float* ytl = yth + h * r;
+    float* x22h = ytl + h * r;
+    float* x22l = x22h + r * r;
+    split_tf32(c, Y, r, h, h, yth, ytl, r, true);
+    split_tf32(c, X22, r, r, ld, x22h, x22l, r);
+    // X21 = -X22 Y  (A = X22 lower; B stored = Y^T)
+    gemm_tf32x3(c, r, h, r, -1.f, x22h, x22l, r, yth, ytl, r, false, X21, ld, kALower);
+  } else {
+    // X21 = -X22 Y
+    gemm_f32(c, false, false, r, h, r, -1.f, X22, ld, Y, h, 0.f, X21, ld, kALower);
+  }
 }
 
 }  // namespace
+
+size_t factor_split_floats(int64_t n) { return split_need(n) + 4096; }
 
 void launch_diag_stats(const Ctx& c, const float* H, int64_t n, float damp, float hscale,
                        bool fix_dead, DiagStats* stats, unsigned char* dead) {
@@ -271,12 +475,74 @@ void launch_build_reversed(const Ctx& c, const float* H, int64_t n, const int32_
   check_launch("build_reversed_kernel");
 }
 
-void factor_inverse_upper(const Ctx& c, float* M, float* X, float* scratch, float* U, int64_t n) {
+namespace {
+
+void factor_direct(const Ctx& c, float* M, float* X, float* scratch, float* U, int64_t n, float* split) {
   check_cuda(cudaMemsetAsync(X, 0, static_cast<size_t>(n) * n * sizeof(float), c.stream), "memset X");
-  chol_inv_rec(c, M, X, n, 0, n, scratch);
+  chol_inv_rec(c, M, X, n, 0, n, scratch, split);
   const int64_t total = n * n;
   reverse_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, c.stream>>>(X, U, n);
   check_launch("reverse_kernel");
+}
+
+// The factorisation is a fixed sequence of a few hundred small launches for a
+// given n and buffers; it is recorded once into a CUDA graph and replayed.
+struct FactorGraph {
+  int device;
+  int64_t n;
+  const void *M, *X, *scratch, *U, *status, *split;
+  cudaGraphExec_t exec;
+  int64_t launches;
+};
+std::vector<FactorGraph> g_factor_graphs;
+
+}  // namespace
+
+void factor_inverse_upper(const Ctx& c, float* M, float* X, float* scratch, float* U, int64_t n,
+                          bool use_graph, float* split) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (c.stream != nullptr) check_cuda(cudaStreamIsCapturing(c.stream, &cs), "cudaStreamIsCapturing");
+  if (!use_graph || cs != cudaStreamCaptureStatusNone) {
+    factor_direct(c, M, X, scratch, U, n, split);
+    return;
+  }
+  for (const FactorGraph& g : g_factor_graphs) {
+    if (g.device == c.device && g.n == n && g.M == M && g.X == X && g.scratch == scratch && g.U == U &&
+        g.status == c.status && g.split == split) {
+      check_cuda(cudaGraphLaunch(g.exec, c.stream), "cudaGraphLaunch(factor)");
+      count_launches(g.launches);
+      return;
+    }
+  }
+  // Record on a private stream (recording runs nothing), replay on the caller's.
+  static cudaStream_t capture_stream[64] = {};
+  if (capture_stream[c.device & 63] == nullptr)
+    check_cuda(cudaStreamCreateWithFlags(&capture_stream[c.device & 63], cudaStreamNonBlocking),
+               "cudaStreamCreate(capture)");
+  Ctx cc = c;
+  cc.stream = capture_stream[c.device & 63];
+  const int64_t l0 = launch_count();
+  check_cuda(cudaStreamBeginCapture(cc.stream, cudaStreamCaptureModeThreadLocal), "cudaStreamBeginCapture");
+  cudaGraph_t graph = nullptr;
+  try {
+    factor_direct(cc, M, X, scratch, U, n, split);
+  } catch (...) {
+    cudaStreamEndCapture(cc.stream, &graph);
+    if (graph) cudaGraphDestroy(graph);
+    throw;
+  }
+  check_cuda(cudaStreamEndCapture(cc.stream, &graph), "cudaStreamEndCapture");
+  cudaGraphExec_t exec = nullptr;
+  const cudaError_t e = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  check_cuda(e, "cudaGraphInstantiate(factor)");
+  const int64_t recorded = launch_count() - l0;
+  if (g_factor_graphs.size() >= 8) {
+    cudaGraphExecDestroy(g_factor_graphs.front().exec);
+    g_factor_graphs.erase(g_factor_graphs.begin());
+  }
+  g_factor_graphs.push_back({c.device, n, M, X, scratch, U, c.status, split, exec, recorded});
+  check_cuda(cudaGraphLaunch(exec, c.stream), "cudaGraphLaunch(factor)");
 }
 
 }  // namespace oc

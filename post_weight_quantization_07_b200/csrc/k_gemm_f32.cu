@@ -135,12 +135,129 @@ __global__ void __launch_bounds__(NT) sgemm_kernel(int64_t M, int64_t N, int64_t
   }
 }
 
+// Small problems (a few tiles): 64x64 tiles for more CTAs and 32-deep k
+// slices so that a product of depth 128-256 takes only a handful of global
+// round trips; 256 threads, 4x4 outputs each.
+constexpr int SM_T = 64, SM_K = 32;
+
+template <bool TA, bool TB>
+__global__ void __launch_bounds__(256) sgemm_small_kernel(int64_t M, int64_t N, int64_t K, float alpha,
+                                                          const float* __restrict__ A, int64_t lda,
+                                                          const float* __restrict__ B, int64_t ldb,
+                                                          float beta, float* __restrict__ C, int64_t ldc,
+                                                          unsigned flags) {
+  const int64_t i0 = static_cast<int64_t>(blockIdx.y) * SM_T;
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x) * SM_T;
+  if ((flags & kCLowerOnly) && j0 > i0 + SM_T - 1) return;
+  int64_t kb = 0, ke = K;
+  if (flags & kAUpper) kb = max(kb, i0);
+  if (flags & kALower) ke = min(ke, i0 + SM_T);
+  if (flags & kBLower) kb = max(kb, j0);
+  if (flags & kBUpper) ke = min(ke, j0 + SM_T);
+
+  __shared__ __align__(16) float As[2][SM_K][SM_T + 4];
+  __shared__ __align__(16) float Bs[2][SM_K][SM_T + 4];
+  const int t = threadIdx.x;
+  const int tx = t & 15, ty = t >> 4;
+  float ra[8], rb[8];
+  auto load = [&](int64_t k0) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int idx = t + 256 * e;  // 0..2047 over a 64 x 32 slice
+      int64_t i, k, j;
+      if (TA) {  // A stored K x M: rows k, contiguous i
+        k = k0 + idx / SM_T;
+        i = i0 + idx % SM_T;
+        ra[e] = (i < M && k < ke) ? A[k * lda + i] : 0.f;
+      } else {
+        i = i0 + idx / SM_K;
+        k = k0 + idx % SM_K;
+        ra[e] = (i < M && k < ke) ? A[i * lda + k] : 0.f;
+      }
+      if (TB) {  // B stored N x K
+        j = j0 + idx / SM_K;
+        k = k0 + idx % SM_K;
+        rb[e] = (j < N && k < ke) ? B[j * ldb + k] : 0.f;
+      } else {
+        k = k0 + idx / SM_T;
+        j = j0 + idx % SM_T;
+        rb[e] = (j < N && k < ke) ? B[k * ldb + j] : 0.f;
+      }
+    }
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int idx = t + 256 * e;
+      if (TA) As[buf][idx / SM_T][idx % SM_T] = ra[e];
+      else As[buf][idx % SM_K][idx / SM_K] = ra[e];
+      if (TB) Bs[buf][idx % SM_K][idx / SM_K] = rb[e];
+      else Bs[buf][idx / SM_T][idx % SM_T] = rb[e];
+    }
+  };
+  float acc[4][4] = {};
+  if (kb < ke) {
+    load(kb);
+    store(0);
+    __syncthreads();
+    int buf = 0;
+    for (int64_t k0 = kb; k0 < ke; k0 += SM_K) {
+      const bool more = k0 + SM_K < ke;
+      if (more) load(k0 + SM_K);
+#pragma unroll 8
+      for (int kk = 0; kk < SM_K; ++kk) {
+        const float4 a4 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+        const float4 b4 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+        const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+      }
+      if (more) {
+        store(buf ^ 1);
+        __syncthreads();
+        buf ^= 1;
+      }
+    }
+  }
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    const int64_t i = i0 + ty * 4 + x;
+    if (i >= M) continue;
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const int64_t j = j0 + tx * 4 + y;
+      if (j >= N) continue;
+      float v = alpha * acc[x][y];
+      if (beta != 0.f) v = fmaf(beta, C[i * ldc + j], v);
+      C[i * ldc + j] = v;
+    }
+  }
+}
+
 }  // namespace
 
 void gemm_f32(const Ctx& c, bool tA, bool tB, int64_t M, int64_t N, int64_t K, float alpha,
               const float* A, int64_t lda, const float* B, int64_t ldb, float beta, float* C,
               int64_t ldc, unsigned flags) {
   if (M <= 0 || N <= 0) return;
+  const int64_t big_tiles = ((M + TM - 1) / TM) * ((N + TN - 1) / TN);
+  if (big_tiles < 2 * static_cast<int64_t>(c.sm_count)) {
+    dim3 grid(static_cast<unsigned>((N + SM_T - 1) / SM_T), static_cast<unsigned>((M + SM_T - 1) / SM_T));
+    if (grid.y > 65535u) fail(OC_ERR_INVALID_ARG, "gemm_f32: M too large");
+    if (!tA && !tB)
+      sgemm_small_kernel<false, false><<<grid, 256, 0, c.stream>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, flags);
+    else if (!tA && tB)
+      sgemm_small_kernel<false, true><<<grid, 256, 0, c.stream>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, flags);
+    else if (tA && !tB)
+      sgemm_small_kernel<true, false><<<grid, 256, 0, c.stream>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, flags);
+    else
+      sgemm_small_kernel<true, true><<<grid, 256, 0, c.stream>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc, flags);
+    check_launch("sgemm_small_kernel");
+    return;
+  }
   dim3 grid(static_cast<unsigned>((N + TN - 1) / TN), static_cast<unsigned>((M + TM - 1) / TM));
   if (grid.y > 65535u) fail(OC_ERR_INVALID_ARG, "gemm_f32: M too large");
   if (!tA && !tB)

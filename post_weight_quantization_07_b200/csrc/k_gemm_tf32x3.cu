@@ -45,6 +45,12 @@ struct Params {
   int* status;
 };
 
+// Tiles wholly above the diagonal are skipped when only the lower triangle of
+// C is wanted (every role applies the same test, so the pipelines stay aligned).
+__device__ __forceinline__ bool tile_skipped(const Params& p, int i0, int j0) {
+  return (p.flags & kCLowerOnly) && j0 > i0 + BM - 1;
+}
+
 __device__ __forceinline__ void k_range(const Params& p, int i0, int j0, int& kb, int& ke) {
   kb = 0;
   ke = p.K;
@@ -110,6 +116,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constan
     bool ok = true;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
       const int i0 = (t % p.tiles_m) * BM, j0 = (t / p.tiles_m) * BN;
+      if (tile_skipped(p, i0, j0)) continue;
       int kb, ke;
       k_range(p, i0, j0, kb, ke);
       for (int k0 = kb; k0 < ke; k0 += BK) {
@@ -151,8 +158,9 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constan
     uint64_t consumed = 0;
     int it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
       const int i0 = (t % p.tiles_m) * BM, j0 = (t / p.tiles_m) * BN;
+      if (tile_skipped(p, i0, j0)) continue;
       int kb, ke;
       k_range(p, i0, j0, kb, ke);
       const int acc = it & 1;
@@ -192,6 +200,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constan
       if (!ok) break;
       if (lane == 0) mma_commit(&tfull[acc]);
       __syncwarp();
+      ++it;
     }
     if (lane == 0) {
       if (!ok) {
@@ -208,8 +217,9 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constan
     unsigned char* stage_buf = epi_base + q * 2 * EPI_BOX_BYTES;
     int it = 0, nbuf = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
       const int i0 = (t % p.tiles_m) * BM, j0 = (t / p.tiles_m) * BN;
+      if (tile_skipped(p, i0, j0)) continue;
       int kb, ke;
       k_range(p, i0, j0, kb, ke);
       const bool empty_k = kb >= ke;
@@ -256,6 +266,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+      ++it;
     }
     if (!ok && lane == 0) {
       record_error(p.status, kDevTimeout);

@@ -290,6 +290,7 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
     sizing.take<float>(mn);                       // W_hi -> G_hi -> T_hi
     sizing.take<float>(mn);                       // W_lo -> G_lo -> T_lo
     sizing.take<float>(mn);                       // G -> T
+    sizing.take<float>(factor_split_floats(n));   // split copies inside the factorisation
     sizing.take<DiagStats>(1);
     Carve cv{workspace(c, sizing.off + 256)};
     float* D = cv.take<float>(nn);
@@ -301,6 +302,7 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
     float* Ph = cv.take<float>(mn);
     float* Pl = cv.take<float>(mn);
     float* G = cv.take<float>(mn);
+    float* fsplit = cv.take<float>(factor_split_floats(n));
     DiagStats* stats = cv.take<DiagStats>(1);
 
     // d = X^T Xhat - Xhat^T Xhat  (the second term from H = 2 Xhat^T Xhat)
@@ -330,7 +332,7 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
       PhaseScope ps(c, kPhFactor);
       launch_diag_stats(c, Hp, n, damp, 1.0f, false, stats, nullptr);
       launch_build_reversed(c, Hp, n, nullptr, stats, 1.0f, false, D);
-      factor_inverse_upper(c, D, Xi, scratch, D, n);
+      factor_inverse_upper(c, D, Xi, scratch, D, n, true, fsplit);
     }
     {
       // W_out = W + alpha G A^-1 = W + 2 alpha (G U^T) U
@@ -383,6 +385,7 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
     sizing.take<float>(static_cast<size_t>(m) * 128);  // Err_lo
     sizing.take<int32_t>(2 * static_cast<size_t>(n));  // perm | inverse
     sizing.take<unsigned char>(n);     // dead
+    sizing.take<float>(factor_split_floats(n));  // split copies inside the factorisation
     sizing.take<DiagStats>(1);
     Carve cv{workspace(c, sizing.off + 256)};
     float* M = cv.take<float>(nn);
@@ -395,6 +398,7 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
     float* Errl = cv.take<float>(static_cast<size_t>(m) * 128);
     int32_t* perm = cv.take<int32_t>(2 * static_cast<size_t>(n));
     unsigned char* dead = cv.take<unsigned char>(n);
+    float* fsplit = cv.take<float>(factor_split_floats(n));
     DiagStats* stats = cv.take<DiagStats>(1);
 
     {
@@ -403,7 +407,7 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
       if (act_order) launch_act_order_perm(c, H, n, perm);
       else launch_identity_perm(c, n, perm);
       launch_build_reversed(c, H, n, perm, stats, 1.0f, true, M);
-      factor_inverse_upper(c, M, Xi, scratch, M, n);
+      factor_inverse_upper(c, M, Xi, scratch, M, n, true, fsplit);
     }
     const float* U = M;
     float* UTh = Xi;

@@ -58,6 +58,7 @@ enum Phase : int {
 };
 
 void count_launch();
+void count_launches(int64_t k);  // launches replayed from a recorded graph
 int64_t launch_count();
 void profile_enable(bool on);
 int profile_read(double* ms, int64_t* launches, int max_phases);
@@ -131,8 +132,13 @@ void gemm_tf32x3(const Ctx& c, int64_t M, int64_t N, int64_t K, float alpha, con
 // U = upper Cholesky factor of (H_prepared)^-1, where H_prepared is formed by
 // `launch_build_reversed` into M (consumed).  Scratch must hold n*n/2 + 4096
 // floats.  X receives L^-1 of the reversed matrix (lower), U its reversal.
+// use_graph: record the launch sequence once per (n, buffers) into a CUDA
+// graph and replay it (instantiating a graph allocates; pass false to run the
+// launches directly).  split: NULL, or room for factor_split_floats(n) floats,
+// which lets the large products run on the tensor cores (3xTF32).
 void factor_inverse_upper(const Ctx& c, float* M, float* X, float* scratch, float* U,
-                          int64_t n);
+                          int64_t n, bool use_graph = true, float* split = nullptr);
+size_t factor_split_floats(int64_t n);
 
 // M[a][b] = Hfix[p(n-1-a)][p(n-1-b)] + lam*[a==b] where Hfix has dead
 // diagonal entries set to 1 (when fix_dead), p = perm (identity if null) and

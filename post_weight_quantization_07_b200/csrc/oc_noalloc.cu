@@ -128,7 +128,7 @@ int run(const float* W, int64_t m, int64_t n, const float* H, int wbits, int gro
   if (act_order) launch_act_order_perm(c, H, n, perm);
   else launch_identity_perm(c, n, perm);
   launch_build_reversed(c, H, n, perm, stats, 1.0f, true, M);
-  factor_inverse_upper(c, M, Xi, scratch, M, n);
+  factor_inverse_upper(c, M, Xi, scratch, M, n, /*use_graph=*/false);  // no graph: it would allocate
   const float* U = M;
   launch_permute_w(c, W, m, n, perm, dead, Wp);
   if (act_order) launch_static_grid(c, W, m, n, static_cast<int>(G), wbits, dead, scales, zeros);

@@ -40,6 +40,8 @@ cudaEvent_t take_event() {
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+void count_launches(int64_t k) { g_launches.fetch_add(k, std::memory_order_relaxed); }
+
 PhaseScope::PhaseScope(const Ctx& c, Phase p) : stream_(c.stream), phase_(p) {
   if (!g_on) return;
   a_ = take_event();
