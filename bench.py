@@ -2,8 +2,11 @@
 """Benchmark: GPTQ+QEP layers quantised per second on one Llama-2-7B-shaped layer.
 
 One step = the whole per-layer path on one synthetic layer already resident in
-HBM: H = 2 Xhat^T Xhat (oc_hessian_accumulate), the QEP correction
-(oc_qep_correct with that H) and GPTQ with packing (oc_gptq_quantize).
+HBM: H = 2 Xhat^T Xhat, the QEP correction with that H and GPTQ with packing,
+through the library's one-call layer entry point (oc_quantize_layer, one
+factorisation of the dampened Hessian).  The same layer through the three
+separate calls (oc_hessian_accumulate, oc_qep_correct, oc_gptq_quantize) is
+timed as well and reported beside it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -125,7 +128,7 @@ def gpu_index_for(local_rank):
 
 # ----------------------------------------------------------------------------- algorithmic work
 
-def phase_work(spec):
+def phase_work(spec, factorisations=1):
     """Algorithmic work of each phase of one layer: (amount, unit, bound)."""
     n, m, N = spec.d_in, spec.d_out, spec.n_tok
     G = spec.d_in if spec.groupsize == -1 else spec.groupsize
@@ -135,8 +138,8 @@ def phase_work(spec):
         "hessian_syrk": (n * (n + 1) * N, "flop", "tensor"),
         "qep_cross": (2 * n * n * N, "flop", "tensor"),
         "qep_w_delta": (2 * m * n * n, "flop", "f32"),
-        # one Cholesky (n^3/3) + one triangular inverse (n^3/3), for QEP and again for GPTQ
-        "factor": (2 * (2 * n ** 3 // 3), "flop", "f32"),
+        # per factorisation one Cholesky (n^3/3) + one triangular inverse (n^3/3)
+        "factor": (factorisations * (2 * n ** 3 // 3), "flop", "f32"),
         "qep_apply": (2 * m * n * n, "flop", "f32"),
         "gptq_trailing": (trailing, "flop", "f32"),
         # read W (fp32) once, write codes (u8) and block errors (fp32)
@@ -248,6 +251,11 @@ def run_ours(args, rank, world, local_rank):
     oc.oc_set_sync(False)
 
     def step():
+        oc.oc_quantize_layer(W, X, Xh, spec.alpha, spec.damp, spec.wbits, spec.groupsize,
+                             spec.act_order, H=H, W_out=Wp, codes=codes, scales=scales,
+                             zeros=zeros, stream=stream)
+
+    def step_three_calls():
         H.zero_()
         oc.oc_hessian_accumulate(Xh, H, stream=stream)
         oc.oc_qep_correct(W, X, Xh, spec.alpha, spec.damp, H_opt=H, W_out=Wp, stream=stream)
@@ -294,6 +302,20 @@ def run_ours(args, rank, world, local_rank):
     ms_total = max_over_ranks(e0.elapsed_time(e1))
     ms_per_step = ms_total / args.steps
     value = world * args.steps / (ms_total / 1e3)
+
+    # ---- the same layer through the three separate calls (two factorisations)
+    step_three_calls()
+    barrier()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(args.steps):
+        step_three_calls()
+    g1.record(stream)
+    barrier()
+    st = oc.oc_stream_status(stream)
+    if st != oc.OC_OK:
+        raise RuntimeError(f"three-call steps failed: {oc.oc_status_string(st)}")
+    ms_three = max_over_ranks(g0.elapsed_time(g1)) / args.steps
 
     # ---- end to end: pinned host inputs copied in and results read back every step
     e2e = None
@@ -404,6 +426,7 @@ def run_ours(args, rank, world, local_rank):
                        parallelism=(f"{world} independent layers, one per rank" if world > 1
                                     else "single GPU")),
         "seconds_per_224_layers_of_this_shape": round(224 * ms_per_step / 1e3, 3),
+        "three_calls_ms_per_step": round(ms_three, 3),
         "layer_roofline_ms_current_units": round(t_roof * 1e3, 3),
         "roofline": roof, "phases": phase_out, "gpu_launches": int(launches),
         "clocks": clocks, "e2e": e2e,

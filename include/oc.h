@@ -181,6 +181,29 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
                      float* scales, float* zeros, int32_t* perm_out, void* stream);
 
 /*
+ * One layer end to end (the OneComp pipeline's GPTQ + QEP step for one linear
+ * layer, OneComp release summary section "量化錯誤傳播 (QEP)" and One
+ * Compression hub page section "核心功能拆解"):
+ *   H      = 2 Xhat^T Xhat                                (overwritten),
+ *   W_out  = W + alpha W d A^-1  as oc_qep_correct with H_opt = H,
+ *   codes, scales, zeros, perm_out = GPTQ of W_out with H as oc_gptq_quantize.
+ * Same results as the three calls in sequence (within rounding), with less
+ * work: GPTQ's dampened Hessian H + damp mean(diag H) I equals QEP's 2A when
+ * no column is dead, so one factorisation serves both (QEP is applied in
+ * GPTQ's processing order).  With dead columns the two dampening constants
+ * differ and two factorisations are made.  The call reads the dead-column
+ * count back to the host once (a short synchronisation of its stream).
+ *   W         fp32 [m x n], read only.    X, Xhat  bf16 [n_tok x n].
+ *   H         fp32 [n x n], written.      W_out    fp32 [m x n], written; must not alias W.
+ *   wbits, groupsize, damp, act_order, codes, scales, zeros, perm_out:
+ *             as oc_gptq_quantize.        alpha: as oc_qep_correct.
+ */
+int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const void* Xhat,
+                      int64_t n_tok, float alpha, float damp, int wbits, int groupsize,
+                      int act_order, float* H, float* W_out, uint32_t* codes, float* scales,
+                      float* zeros, int32_t* perm_out, void* stream);
+
+/*
  * Allocation-free GPTQ (no counterpart in the paper: an addition for callers of
  * this library).  Some callers cannot have a library allocate device memory on
  * its own -- e.g. a process whose memory is entirely reserved for its own

@@ -19,7 +19,7 @@ __all__ = ["OC_OK", "OC_ERR_INVALID_ARG", "OC_ERR_UNSUPPORTED", "OC_ERR_NOT_SPD"
            "LIB_PATH", "HEADER_PATH", "lib", "declared_symbols", "oc_hessian_accumulate",
            "oc_qep_correct", "oc_gptq_quantize", "oc_set_sync", "oc_stream_status",
            "oc_workspace_release", "oc_status_string", "oc_last_error", "oc_version",
-           "oc_profile_enable", "oc_profile_read", "oc_launch_count"]
+           "oc_profile_enable", "oc_profile_read", "oc_launch_count", "oc_quantize_layer"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liboc.so")
@@ -76,6 +76,9 @@ def _load():
     L.oc_qep_correct.restype = i32
     L.oc_gptq_quantize.argtypes = [vp, i64, i64, vp, i32, i32, f32, i32, vp, vp, vp, vp, vp]
     L.oc_gptq_quantize.restype = i32
+    L.oc_quantize_layer.argtypes = [vp, i64, i64, vp, vp, i64, f32, f32, i32, i32, i32, vp, vp, vp, vp,
+                                    vp, vp, vp]
+    L.oc_quantize_layer.restype = i32
     return L
 
 
@@ -228,3 +231,36 @@ def oc_gptq_quantize(W, H, wbits, groupsize, damp, act_order, codes=None, scales
                               _stream_handle(stream))
     _check(st, "oc_gptq_quantize")
     return codes, scales, zeros, perm_out
+
+
+def oc_quantize_layer(W, X, Xhat, alpha, damp, wbits, groupsize, act_order, H=None, W_out=None,
+                      codes=None, scales=None, zeros=None, perm_out=None, stream=None):
+    """Hessian + QEP + GPTQ of one layer in one call (one factorisation when no
+    column is dead).  Returns (H, W_out, codes, scales, zeros, perm_out)."""
+    import torch
+    m, n = W.shape
+    n_tok = X.shape[0]
+    G = n if groupsize == -1 else int(groupsize)
+    ng = max(1, n // G)
+    dev = W.device
+    if H is None:
+        H = torch.empty(n, n, dtype=torch.float32, device=dev)
+    if W_out is None:
+        W_out = torch.empty_like(W)
+    if codes is None:
+        codes = torch.empty(m, n * wbits // 32, dtype=torch.int32, device=dev)
+    if scales is None:
+        scales = torch.empty(m, ng, dtype=torch.float32, device=dev)
+    if zeros is None:
+        zeros = torch.empty(m, ng, dtype=torch.float32, device=dev)
+    pp = _dev_ptr(perm_out, torch.int32, "perm_out", (n,)) if perm_out is not None else None
+    st = _lib().oc_quantize_layer(
+        _dev_ptr(W, torch.float32, "W"), m, n, _dev_ptr(X, torch.bfloat16, "X", (n_tok, n)),
+        _dev_ptr(Xhat, torch.bfloat16, "Xhat", (n_tok, n)), n_tok, float(alpha), float(damp),
+        int(wbits), int(groupsize), 1 if act_order else 0, _dev_ptr(H, torch.float32, "H", (n, n)),
+        _dev_ptr(W_out, torch.float32, "W_out", (m, n)),
+        _dev_ptr(codes, torch.int32, "codes", (m, n * wbits // 32)),
+        _dev_ptr(scales, torch.float32, "scales", (m, ng)),
+        _dev_ptr(zeros, torch.float32, "zeros", (m, ng)), pp, _stream_handle(stream))
+    _check(st, "oc_quantize_layer")
+    return H, W_out, codes, scales, zeros, perm_out

@@ -156,6 +156,7 @@ struct LeafSmem {
   float T[(LEAF / 2) * LDT];       // L21 of the 128 level; temporaries of the 64 level
   float Y[(LEAF / 2) * LDT];       // Y of the 128 level (lives across the right half)
   float L32[32 * 33];              // factor of the current 32 block
+  float R32[32];                   // reciprocals of its diagonal
 };
 
 __device__ __forceinline__ void warp_chol_inv32(LeafSmem& sm, int off, int* status) {
@@ -178,20 +179,29 @@ __device__ __forceinline__ void warp_chol_inv32(LeafSmem& sm, int off, int* stat
     }
   }
   if (bad && lane == 0) record_error(status, kDevNotSpd);
+  float dl = 1.f;
 #pragma unroll
-  for (int j = 0; j < 32; ++j) sm.L32[lane * 33 + j] = a[j];
+  for (int j = 0; j < 32; ++j) {
+    sm.L32[lane * 33 + j] = a[j];
+    if (j == lane) dl = a[j];
+  }
+  sm.R32[lane] = 1.f / dl;
   __syncwarp();
-  // column `lane` of X = L^-1: x_i = (delta_i,lane - sum_{k<i} L_ik x_k) / L_ii
-  float x[32];
+  // Column `lane` of X = L^-1 by right-looking forward substitution: at step k
+  // x_k = b_k / L_kk, then every later row takes b_i -= L_ik x_k (independent
+  // updates: the dependent chain is one multiply and one FMA per step).
+  float b[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    float acc = (i == lane) ? 1.f : 0.f;
+  for (int i = 0; i < 32; ++i) b[i] = (i == lane) ? 1.f : 0.f;
 #pragma unroll
-    for (int k = 0; k < i; ++k) acc = fmaf(-sm.L32[i * 33 + k], x[k], acc);
-    x[i] = acc / sm.L32[i * 33 + i];
+  for (int k = 0; k < 32; ++k) {
+    const float xk = b[k] * sm.R32[k];
+    b[k] = xk;
+#pragma unroll
+    for (int i = k + 1; i < 32; ++i) b[i] = fmaf(-sm.L32[i * 33 + k], xk, b[i]);
   }
 #pragma unroll
-  for (int i = 0; i < 32; ++i) sm.X[(off + i) * LDA + off + lane] = x[i];
+  for (int i = 0; i < 32; ++i) sm.X[(off + i) * LDA + off + lane] = b[i];
 }
 
 // The four products of one recursion node of half width H inside the CTA
@@ -314,24 +324,46 @@ __global__ void __launch_bounds__(256) leaf_chol_inv_kernel(const float* __restr
   extern __shared__ __align__(16) float leaf_smem[];
   LeafSmem& sm = *reinterpret_cast<LeafSmem*>(leaf_smem);
   const int t = threadIdx.x;
-  for (int e = t; e < LEAF * LEAF; e += blockDim.x) {
-    const int i = e / LEAF, j = e % LEAF;
-    float v = 0.f;
-    if (j <= i) {
-      if (i < s) v = M[static_cast<int64_t>(i) * ld + j];
-      else if (i == j) v = 1.f;
+  // Load the block with 16 independent 16-byte loads per thread in flight
+  // (rows of M are 16-byte aligned: n is a multiple of 64).
+  float4 v[16];
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int e4 = t + 256 * q;          // float4 index in the 128 x 128 block
+    const int i = e4 >> 5, j = (e4 & 31) * 4;
+    v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < s && j <= i && j < s) v[q] = *reinterpret_cast<const float4*>(M + static_cast<int64_t>(i) * ld + j);
+  }
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int e4 = t + 256 * q;
+    const int i = e4 >> 5, j = (e4 & 31) * 4;
+    const float vv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float x = (j + c <= i && j + c < s) ? vv[c] : 0.f;
+      if (i >= s && i == j + c) x = 1.f;  // identity padding beyond s
+      sm.A[i * LDA + j + c] = x;
+      sm.X[i * LDA + j + c] = 0.f;
     }
-    sm.A[i * LDA + j] = v;
-    sm.X[i * LDA + j] = 0.f;
   }
   __syncthreads();
   leaf64(sm, 0, status);
   node_pre<64>(sm, 0, sm.T, LDT, sm.Y, LDT);
   leaf64(sm, 64, status);
   node_post<64>(sm, 0, sm.Y, LDT);
-  for (int e = t; e < s * s; e += blockDim.x) {
-    const int i = e / s, j = e % s;
-    X[static_cast<int64_t>(i) * ld + j] = (j <= i) ? sm.X[i * LDA + j] : 0.f;
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const int e4 = t + 256 * q;
+    const int i = e4 >> 5, j = (e4 & 31) * 4;
+    if (i < s && j < s) {
+      float4 o;
+      o.x = (j + 0 <= i) ? sm.X[i * LDA + j + 0] : 0.f;
+      o.y = (j + 1 <= i) ? sm.X[i * LDA + j + 1] : 0.f;
+      o.z = (j + 2 <= i) ? sm.X[i * LDA + j + 2] : 0.f;
+      o.w = (j + 3 <= i) ? sm.X[i * LDA + j + 3] : 0.f;
+      *reinterpret_cast<float4*>(X + static_cast<int64_t>(i) * ld + j) = o;
+    }
   }
 }
 

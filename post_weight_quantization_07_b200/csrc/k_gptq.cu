@@ -298,6 +298,11 @@ void launch_pack(const Ctx& c, const unsigned char* codes8, int64_t m, int64_t n
   check_launch("pack_kernel");
 }
 
+void launch_invert_perm(const Ctx& c, int32_t* perm2, int64_t n) {
+  invert_perm_kernel<<<blocks_for(n, 256), 256, 0, c.stream>>>(perm2, n, perm2 + n);
+  check_launch("invert_perm_kernel");
+}
+
 void launch_sub_half(const Ctx& c, float* D, const float* H, int64_t n) {
   sub_half_kernel<<<blocks_for(n * n, 256), 256, 0, c.stream>>>(D, H, n * n);
   check_launch("sub_half_kernel");

@@ -179,6 +179,61 @@ CUtensorMap make_tmap_2d(const void* base, CUtensorMapDataType dt, int elem_byte
 
 }  // namespace oc
 
+namespace oc {
+namespace {
+
+void check_gptq_args(const float* W, int64_t m, int64_t n, int wbits, int groupsize, float damp, int act_order,
+                     const uint32_t* codes, const float* scales, const float* zeros) {
+  if (!W || !codes || !scales || !zeros) fail(OC_ERR_INVALID_ARG, "W, codes, scales, zeros must be non-null");
+  if (n < 64 || n % 64) fail(OC_ERR_INVALID_ARG, "n must be a positive multiple of 64");
+  if (n > 49152) fail(OC_ERR_INVALID_ARG, "n above 49152 is not supported");
+  if (m < 1) fail(OC_ERR_INVALID_ARG, "m must be >= 1");
+  if (wbits < 2 || wbits > 4) fail(OC_ERR_INVALID_ARG, "wbits must be 2, 3 or 4");
+  if (act_order != 0 && act_order != 1) fail(OC_ERR_INVALID_ARG, "act_order must be 0 or 1");
+  if (!(damp >= 0.f) || damp > 3.4e38f) fail(OC_ERR_INVALID_ARG, "damp must be finite and >= 0");
+  const int64_t G = (groupsize == -1) ? n : groupsize;
+  if (G < 4 || n % G) fail(OC_ERR_INVALID_ARG, "groupsize must divide n (or be -1)");
+  const bool pow2_small = G <= 128 && (G & (G - 1)) == 0;
+  if (!(G == n || pow2_small || G % 128 == 0))
+    fail(OC_ERR_INVALID_ARG, "groupsize must be a power of two <= 128, a multiple of 128, or -1");
+  if (!aligned16(codes) || !aligned16(W)) fail(OC_ERR_INVALID_ARG, "W and codes must be 16-byte aligned");
+}
+
+// GPTQ after the factor: blocked sweep over the permuted working copy Wp with
+// tensor-core trailing updates, then packing (and the processing order out).
+void gptq_sweep_and_pack(const Ctx& c, float* Wp, int64_t m, int64_t n, const float* U, const float* UTh,
+                         const float* UTl, int G, int wbits, bool act_order, int32_t* perm, float* scales,
+                         float* zeros, unsigned char* codes8, float* Err, float* Errh, float* Errl, uint32_t* codes,
+                         int32_t* perm_out) {
+  for (int64_t j1 = 0; j1 < n; j1 += 128) {
+    const int64_t bw = std::min<int64_t>(128, n - j1);
+    const int64_t j2 = j1 + bw;
+    {
+      PhaseScope ps(c, kPhGptqSweep);
+      launch_sweep_block(c, Wp, m, n, U, j1, G, wbits, act_order, perm, scales, zeros, codes8, Err);
+    }
+    if (j2 < n) {
+      // W[:, j2:] -= Err U[j1:j2, j2:] on the tensor cores (3xTF32); B stored
+      // = U^T[j2:, j1:j2] (rows j2.., columns j1..j1+bw of the transpose)
+      PhaseScope ps(c, kPhGptqTrailing);
+      split_tf32(c, Err, m, bw, 128, Errh, Errl, 128);
+      gemm_tf32x3(c, m, n - j2, bw, -1.f, Errh, Errl, 128, UTh + j2 * n + j1, UTl + j2 * n + j1, n, true, Wp + j2,
+                  n, kANone);
+    }
+  }
+  {
+    PhaseScope ps(c, kPhGptqPack);
+    launch_pack(c, codes8, m, n, wbits, perm, codes);
+  }
+  if (perm_out)
+    check_cuda(cudaMemcpyAsync(perm_out, perm, static_cast<size_t>(n) * sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                               c.stream),
+               "copy perm");
+}
+
+}  // namespace
+}  // namespace oc
+
 using namespace oc;
 
 extern "C" {
@@ -359,19 +414,9 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
                      int act_order, uint32_t* codes, float* scales, float* zeros, int32_t* perm_out,
                      void* stream) {
   return guarded([&]() -> int {
-    if (!W || !H || !codes || !scales || !zeros) fail(OC_ERR_INVALID_ARG, "W, H, codes, scales, zeros must be non-null");
-    if (n < 64 || n % 64) fail(OC_ERR_INVALID_ARG, "n must be a positive multiple of 64");
-    if (n > 49152) fail(OC_ERR_INVALID_ARG, "n above 49152 is not supported");
-    if (m < 1) fail(OC_ERR_INVALID_ARG, "m must be >= 1");
-    if (wbits < 2 || wbits > 4) fail(OC_ERR_INVALID_ARG, "wbits must be 2, 3 or 4");
-    if (act_order != 0 && act_order != 1) fail(OC_ERR_INVALID_ARG, "act_order must be 0 or 1");
-    if (!(damp >= 0.f) || damp > 3.4e38f) fail(OC_ERR_INVALID_ARG, "damp must be finite and >= 0");
+    check_gptq_args(W, m, n, wbits, groupsize, damp, act_order, codes, scales, zeros);
+    if (!H) fail(OC_ERR_INVALID_ARG, "H must be non-null");
     const int64_t G = (groupsize == -1) ? n : groupsize;
-    if (G < 4 || n % G) fail(OC_ERR_INVALID_ARG, "groupsize must divide n (or be -1)");
-    const bool pow2_small = G <= 128 && (G & (G - 1)) == 0;
-    if (!(G == n || pow2_small || G % 128 == 0))
-      fail(OC_ERR_INVALID_ARG, "groupsize must be a power of two <= 128, a multiple of 128, or -1");
-    if (!aligned16(codes) || !aligned16(W)) fail(OC_ERR_INVALID_ARG, "W and codes must be 16-byte aligned");
     Ctx c = make_ctx(stream);
     const size_t nn = static_cast<size_t>(n) * n, mn = static_cast<size_t>(m) * n;
     Carve sizing{nullptr};
@@ -418,31 +463,150 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
       launch_permute_w(c, W, m, n, perm, dead, Wp);
       if (act_order) launch_static_grid(c, W, m, n, static_cast<int>(G), wbits, dead, scales, zeros);
     }
-    for (int64_t j1 = 0; j1 < n; j1 += 128) {
-      const int64_t bw = std::min<int64_t>(128, n - j1);
-      const int64_t j2 = j1 + bw;
-      {
-        PhaseScope ps(c, kPhGptqSweep);
-        launch_sweep_block(c, Wp, m, n, U, j1, static_cast<int>(G), wbits, act_order != 0, perm, scales, zeros,
-                           codes8, Err);
-      }
-      if (j2 < n) {
-        // W[:, j2:] -= Err U[j1:j2, j2:] on the tensor cores (3xTF32)
-        PhaseScope ps(c, kPhGptqTrailing);
-        split_tf32(c, Err, m, bw, 128, Errh, Errl, 128);
-        // B stored = U^T[j2:, j1:j2] (rows j2.., columns j1..j1+bw of the transpose)
-        gemm_tf32x3(c, m, n - j2, bw, -1.f, Errh, Errl, 128, UTh + j2 * n + j1, UTl + j2 * n + j1, n, true,
-                    Wp + j2, n, kANone);
-      }
+    gptq_sweep_and_pack(c, Wp, m, n, U, UTh, UTl, static_cast<int>(G), wbits, act_order != 0, perm, scales, zeros,
+                        codes8, Err, Errh, Errl, codes, perm_out);
+    return finish(c);
+  });
+}
+
+int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const void* Xhat, int64_t n_tok,
+                      float alpha, float damp, int wbits, int groupsize, int act_order, float* H, float* W_out,
+                      uint32_t* codes, float* scales, float* zeros, int32_t* perm_out, void* stream) {
+  return guarded([&]() -> int {
+    check_gptq_args(W, m, n, wbits, groupsize, damp, act_order, codes, scales, zeros);
+    if (!X || !Xhat || !H || !W_out) fail(OC_ERR_INVALID_ARG, "X, Xhat, H, W_out must be non-null");
+    if (W_out == W) fail(OC_ERR_INVALID_ARG, "W_out must not alias W");
+    if (n_tok < 1 || n_tok > (int64_t(1) << 31) - 64) fail(OC_ERR_INVALID_ARG, "n_tok out of range");
+    if (!(alpha == alpha) || alpha > 3.4e38f || alpha < -3.4e38f) fail(OC_ERR_INVALID_ARG, "alpha must be finite");
+    if (!aligned16(X) || !aligned16(Xhat) || !aligned16(H) || !aligned16(W_out))
+      fail(OC_ERR_INVALID_ARG, "X, Xhat, H, W_out must be 16-byte aligned");
+    const int64_t G = (groupsize == -1) ? n : groupsize;
+    Ctx c = make_ctx(stream);
+    const size_t nn = static_cast<size_t>(n) * n, mn = static_cast<size_t>(m) * n;
+    Carve sizing{nullptr};
+    sizing.take<float>(nn);                 // d -> M -> U
+    sizing.take<float>(nn);                 // d^T hi -> inverse factor -> U hi
+    sizing.take<float>(nn + 4096);          // d^T lo -> recursion scratch -> U lo
+    sizing.take<float>(nn);                 // U^T hi
+    sizing.take<float>(nn);                 // U^T lo
+    sizing.take<float>(mn);                 // hi halves (W, G, T)
+    sizing.take<float>(mn);                 // lo halves
+    sizing.take<float>(mn);                 // G -> T
+    sizing.take<float>(mn);                 // permuted working copy of W
+    sizing.take<unsigned char>(mn);         // codes, processing order
+    sizing.take<float>(3 * static_cast<size_t>(m) * 128);  // block errors and their halves
+    sizing.take<int32_t>(2 * static_cast<size_t>(n));      // order | inverse
+    sizing.take<unsigned char>(n);          // dead-column mask
+    sizing.take<float>(factor_split_floats(n));
+    sizing.take<DiagStats>(1);
+    Carve cv{workspace(c, sizing.off + 256)};
+    float* D = cv.take<float>(nn);
+    float* Xi = cv.take<float>(nn);
+    float* scratch = cv.take<float>(nn + 4096);
+    float* UTh = cv.take<float>(nn);
+    float* UTl = cv.take<float>(nn);
+    float* Ph = cv.take<float>(mn);
+    float* Pl = cv.take<float>(mn);
+    float* G2 = cv.take<float>(mn);
+    float* Wp = cv.take<float>(mn);
+    unsigned char* codes8 = cv.take<unsigned char>(mn);
+    float* Err = cv.take<float>(3 * static_cast<size_t>(m) * 128);
+    float* Errh = Err + static_cast<size_t>(m) * 128;
+    float* Errl = Errh + static_cast<size_t>(m) * 128;
+    int32_t* perm = cv.take<int32_t>(2 * static_cast<size_t>(n));
+    unsigned char* dead = cv.take<unsigned char>(n);
+    float* fsplit = cv.take<float>(factor_split_floats(n));
+    DiagStats* stats = cv.take<DiagStats>(1);
+
+    {
+      PhaseScope ps(c, kPhHessian);
+      check_cuda(cudaMemsetAsync(H, 0, nn * sizeof(float), c.stream), "memset H");
+      launch_atb_bf16(c, Xhat, Xhat, n_tok, n, n, 2.0f, H, n, true);
+      launch_mirror_upper(c, H, n);
     }
     {
-      PhaseScope ps(c, kPhGptqPack);
-      launch_pack(c, codes8, m, n, wbits, perm, codes);
+      PhaseScope ps(c, kPhQepCross);
+      check_cuda(cudaMemsetAsync(D, 0, nn * sizeof(float), c.stream), "memset d");
+      launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false);
+      launch_sub_half(c, D, H, n);
     }
-    if (perm_out)
-      check_cuda(cudaMemcpyAsync(perm_out, perm, static_cast<size_t>(n) * sizeof(int32_t), cudaMemcpyDeviceToDevice,
-                                 c.stream),
-                 "copy perm");
+    {
+      PhaseScope ps(c, kPhQepWDelta);
+      split_tf32(c, D, n, n, n, Xi, scratch, n, true);
+      split_tf32(c, W, m, n, n, Ph, Pl, n);
+      gemm_tf32x3(c, m, n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, G2, n, kANone);
+    }
+    // GPTQ's dampened Hessian equals QEP's 2A unless a column is dead (their
+    // dampening constants then differ): one device-to-host read decides.
+    launch_diag_stats(c, H, n, damp, 1.0f, true, stats, dead);
+    DiagStats hs{};
+    check_cuda(cudaMemcpyAsync(&hs, stats, sizeof(DiagStats), cudaMemcpyDeviceToHost, c.stream), "read stats");
+    check_cuda(cudaStreamSynchronize(c.stream), "cudaStreamSynchronize");
+    if (hs.nonfinite) return finish(c);
+    if (hs.n_dead > 0) {
+      // two factorisations: QEP's own (original order), then GPTQ's
+      {
+        PhaseScope ps(c, kPhFactor);
+        DiagStats* qs = stats;
+        launch_diag_stats(c, H, n, damp, 1.0f, false, qs, nullptr);
+        launch_build_reversed(c, H, n, nullptr, qs, 1.0f, false, D);
+        factor_inverse_upper(c, D, Xi, scratch, D, n, true, fsplit);
+      }
+      {
+        PhaseScope ps(c, kPhQepApply);
+        split_tf32(c, D, n, n, n, Xi, scratch, n);
+        split_tf32(c, D, n, n, n, UTh, UTl, n, true);
+        split_tf32(c, G2, m, n, n, Ph, Pl, n);
+        gemm_tf32x3(c, m, n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, G2, n, kBLower);
+        split_tf32(c, G2, m, n, n, Ph, Pl, n);
+        launch_copy_f32(c, W, W_out, static_cast<int64_t>(mn));
+        gemm_tf32x3(c, m, n, n, 2.f * alpha, Ph, Pl, n, UTh, UTl, n, true, W_out, n, kBUpper);
+      }
+      {
+        PhaseScope ps(c, kPhFactor);
+        launch_diag_stats(c, H, n, damp, 1.0f, true, stats, dead);
+        if (act_order) launch_act_order_perm(c, H, n, perm);
+        else launch_identity_perm(c, n, perm);
+        launch_build_reversed(c, H, n, perm, stats, 1.0f, true, D);
+        factor_inverse_upper(c, D, Xi, scratch, D, n, true, fsplit);
+      }
+      {
+        PhaseScope ps(c, kPhGptqPrep);
+        split_tf32(c, D, n, n, n, UTh, UTl, n, true);
+        launch_permute_w(c, W_out, m, n, perm, dead, Wp);
+        if (act_order) launch_static_grid(c, W_out, m, n, static_cast<int>(G), wbits, dead, scales, zeros);
+      }
+    } else {
+      // one factorisation of P H_d P^T; QEP applied in processing order:
+      //   W'P = WP + 2 alpha ((G P) U^T) U
+      {
+        PhaseScope ps(c, kPhFactor);
+        if (act_order) launch_act_order_perm(c, H, n, perm);
+        else launch_identity_perm(c, n, perm);
+        launch_build_reversed(c, H, n, perm, stats, 1.0f, true, D);
+        factor_inverse_upper(c, D, Xi, scratch, D, n, true, fsplit);
+      }
+      {
+        PhaseScope ps(c, kPhQepApply);
+        const float* U = D;
+        split_tf32(c, U, n, n, n, Xi, scratch, n);
+        split_tf32(c, U, n, n, n, UTh, UTl, n, true);
+        launch_permute_w(c, G2, m, n, perm, dead, Wp);           // G P
+        split_tf32(c, Wp, m, n, n, Ph, Pl, n);
+        gemm_tf32x3(c, m, n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, G2, n, kBLower);  // T = (G P) U^T
+        split_tf32(c, G2, m, n, n, Ph, Pl, n);
+        launch_permute_w(c, W, m, n, perm, dead, Wp);            // W P
+        gemm_tf32x3(c, m, n, n, 2.f * alpha, Ph, Pl, n, UTh, UTl, n, true, Wp, n, kBUpper);
+        launch_invert_perm(c, perm, n);
+        launch_permute_w(c, Wp, m, n, perm + n, dead, W_out);    // back to original order
+      }
+      if (act_order) {
+        PhaseScope ps(c, kPhGptqPrep);
+        launch_static_grid(c, W_out, m, n, static_cast<int>(G), wbits, dead, scales, zeros);
+      }
+    }
+    gptq_sweep_and_pack(c, Wp, m, n, D, UTh, UTl, static_cast<int>(G), wbits, act_order != 0, perm, scales, zeros,
+                        codes8, Err, Errh, Errl, codes, perm_out);
     return finish(c);
   });
 }

@@ -170,6 +170,9 @@ void launch_sweep_block(const Ctx& c, float* Wp, int64_t m, int64_t n, const flo
 void launch_pack(const Ctx& c, const unsigned char* codes8, int64_t m, int64_t n, int wbits,
                  int32_t* perm2, uint32_t* codes);
 
+// perm2[n .. 2n) := inverse of the permutation in perm2[0 .. n).
+void launch_invert_perm(const Ctx& c, int32_t* perm2, int64_t n);
+
 // QEP pieces.
 void launch_sub_half(const Ctx& c, float* D, const float* H, int64_t n);  // D -= H/2
 void launch_copy_f32(const Ctx& c, const float* src, float* dst, int64_t count);

@@ -286,3 +286,37 @@ def test_end_to_end_512_workload():
     eg = oracle.layer_errors(W, deq, X, Xh)["e_lit"]
     eo = oracle.layer_errors(W, ref["deq"], X, Xh)["e_lit"]
     assert abs(eg - eo) <= 0.01 * eo
+
+
+# ----------------------------------------------------------------------------- fused layer call
+
+@pytest.mark.parametrize("m,n,n_tok,wbits,G,act,dead", [
+    (512, 512, 2048, 4, 128, False, False),
+    (256, 384, 1500, 3, 64, True, False),
+    (96, 256, 1024, 4, 64, True, True),     # dead columns: two factorisations
+    (128, 1024, 4096, 2, 64, True, False),  # large enough for tensor-core factor nodes
+])
+def test_fused_layer_matches_oracle(m, n, n_tok, wbits, G, act, dead):
+    L = random_layer_host(m, n, n_tok, seed=3000 + n + m)
+    W, X, Xh = L["W"].astype(np.float64), L["X"].copy(), L["Xhat"].copy()
+    if dead:
+        X[:, [7, 100]] = 0.0
+        Xh[:, [7, 100]] = 0.0
+    Ho = oracle.hessian(Xh)
+    Wpo = oracle.qep_correct(W, X, Xh, 0.5, 0.01, H=Ho)
+    ref = oracle.gptq_quantize(Wpo, Ho, wbits, G, 0.01, act)
+    perm = torch.empty(n, dtype=torch.int32, device="cuda")
+    Hg, Wpg, codes, scales, zeros, _ = oc.oc_quantize_layer(dev(W), bf16_dev(X), bf16_dev(Xh), 0.5, 0.01,
+                                                            wbits, G, act, perm_out=perm)
+    torch.cuda.synchronize()
+    assert rel_fro(Hg.cpu().numpy(), Ho) <= H_TOL
+    Wpg = Wpg.cpu().numpy()
+    assert np.abs(Wpg - Wpo).max() <= QEP_TOL * np.abs(W).max()
+    cg = oracle.unpack_codes(codes.cpu().numpy().view(np.uint32), wbits, n)
+    sg, zg = scales.cpu().numpy(), zeros.cpu().numpy()
+    pg = perm.cpu().numpy()
+    st = oracle.teacher_forced_check(Wpo, Ho, wbits, G, 0.01, act, cg, sg, zg, perm=pg)
+    assert st["n_bad"] == 0 and st["zero_bad"] == 0, st
+    assert st["scale_max_rel"] <= SCALE_TOL, st
+    ident = level_identity(cg, zg, ref["codes"], ref["zeros"], G)
+    assert ident >= code_frac_for(cg.size), (ident, st)
