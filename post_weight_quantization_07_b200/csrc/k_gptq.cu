@@ -16,7 +16,7 @@ namespace oc {
 namespace {
 
 constexpr int SB = 128;          // sweep block width
-constexpr int SWEEP_WARPS = 16;
+constexpr int SWEEP_WARPS = 4;
 
 __device__ __forceinline__ void grid_from_minmax(float xmin, float xmax, float maxq, float& s,
                                                  float& z) {
@@ -68,130 +68,194 @@ __global__ void static_grid_kernel(const float* __restrict__ W, int64_t m, int64
   }
 }
 
+// 8 lanes per row, 16 consecutive columns per lane (lane q of a row's group
+// holds block columns 16q .. 16q+15), 4 rows per warp.  Step j of the block
+// belongs to lane j / 16 (register j % 16, a compile-time index inside the
+// unrolled 16-step chunk); its error reaches the other 7 lanes of the row by a
+// width-8 shuffle.  Each lane then updates its own later columns from the U
+// row in shared memory.  U rows are stored skewed (4 floats of padding after
+// every 16 columns) so that the 8 lanes' 16-byte reads fall in distinct banks.
+// Groups of 16 columns or more start on chunk boundaries and are handled once
+// per chunk (SMALLG: groups of 4 or 8 columns, checked every step).
+constexpr int LPR = 8;                    // lanes per row
+constexpr int CPL = SB / LPR;             // columns per lane
+constexpr int UPAD = SB + SB / 16 * 4;    // skewed U row length (160 floats)
+__device__ __forceinline__ int upos(int j, int k) { return j * UPAD + k + (k >> 4) * 4; }
+
+template <bool SMALLG>
+__device__ __forceinline__ void group_grid(float (&w)[CPL], float (&sc)[CPL], float (&zc)[CPL], int j, int G,
+                                           int bw, int q, bool g_small, const float* wrow, int64_t j1, float maxq,
+                                           bool store, float* scales, float* zeros, int64_t srow) {
+  float xmin = INFINITY, xmax = -INFINITY;
+  if (g_small) {
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      const int k = CPL * q + i;
+      if (k >= j && k < j + G && k < bw) {
+        xmin = fminf(xmin, w[i]);
+        xmax = fmaxf(xmax, w[i]);
+      }
+    }
+  } else {
+    // a group wider than the block starts at its first column: every column
+    // of it is current (earlier blocks' updates are applied, this block's
+    // have not started)
+    for (int64_t k = j1 + q; k < j1 + G; k += LPR) {
+      const float v = wrow[k];
+      xmin = fminf(xmin, v);
+      xmax = fmaxf(xmax, v);
+    }
+  }
+#pragma unroll
+  for (int o = 1; o < LPR; o <<= 1) {
+    xmin = fminf(xmin, __shfl_xor_sync(0xffffffffu, xmin, o, LPR));
+    xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, o, LPR));
+  }
+  float gs, gz;
+  grid_from_minmax(xmin, xmax, maxq, gs, gz);
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) {
+    const int k = CPL * q + i;
+    if (!g_small || (k >= j && k < j + G)) {
+      sc[i] = gs;
+      zc[i] = gz;
+    }
+  }
+  if (store) {
+    const int64_t g = (j1 + j) / G;
+    scales[srow + g] = gs;
+    zeros[srow + g] = gz;
+  }
+}
+
+template <bool SMALLG>
 __global__ void __launch_bounds__(SWEEP_WARPS * 32)
 sweep_block_kernel(float* __restrict__ Wp, int64_t m, int64_t n, const float* __restrict__ U, int64_t j1, int G,
                    float maxq, int static_groups, const int32_t* __restrict__ perm, float* __restrict__ scales,
                    float* __restrict__ zeros, unsigned char* __restrict__ codes8, float* __restrict__ Err) {
-  extern __shared__ __align__(16) float Ub[];  // [SB][SB]
+  extern __shared__ __align__(16) float Ub[];  // [SB][UPAD], skewed
   const int bw = static_cast<int>(::min((int64_t)SB, n - j1));
-  for (int e = threadIdx.x; e < SB * SB; e += blockDim.x) {
-    const int j = e / SB, k = e % SB;
-    Ub[e] = (j < bw && k < bw) ? U[(j1 + j) * n + j1 + k] : 0.f;
+  {
+    // 16-byte loads, all of a thread's in flight at once (U rows are 16-byte
+    // aligned: n is a multiple of 64); only the upper triangle is non-zero.
+    constexpr int PER = SB * SB / 4 / (SWEEP_WARPS * 32);
+    float4 v[PER];
+#pragma unroll
+    for (int q4 = 0; q4 < PER; ++q4) {
+      const int e4 = threadIdx.x + SWEEP_WARPS * 32 * q4;
+      const int j = e4 / (SB / 4), k = (e4 % (SB / 4)) * 4;
+      v[q4] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j < bw && k < bw && k + 3 >= j) v[q4] = *reinterpret_cast<const float4*>(U + (j1 + j) * n + j1 + k);
+    }
+#pragma unroll
+    for (int q4 = 0; q4 < PER; ++q4) {
+      const int e4 = threadIdx.x + SWEEP_WARPS * 32 * q4;
+      const int j = e4 / (SB / 4), k = (e4 % (SB / 4)) * 4;
+      *reinterpret_cast<float4*>(&Ub[upos(j, k)]) = v[q4];
+    }
   }
   __syncthreads();
+  // reciprocal pivots 1 / U_jj (the serial chain then multiplies instead of dividing)
+  float* rU = Ub + SB * UPAD;
+  if (threadIdx.x < SB) rU[threadIdx.x] = (threadIdx.x < bw) ? 1.f / Ub[upos(threadIdx.x, threadIdx.x)] : 0.f;
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = lane & (LPR - 1);        // lane within the row's group
   const int64_t ng = n / G;
-  const int64_t col0 = j1 + 4 * lane;  // first column of this lane
-  // Group starts inside this block (all 32-bit, no division in the loop): a
-  // group of at most one block (G divides 128) starts wherever j % G == 0; a
-  // wider group can only start at the block's first column.
+  const int64_t col0 = j1 + CPL * q;     // first column of this lane
+  const bool lane_valid = CPL * q < bw;  // bw is 64 or 128
   const bool g_small = G <= SB;
   const bool block_starts_group = (j1 % G) == 0;
-  for (int64_t r = static_cast<int64_t>(blockIdx.x) * SWEEP_WARPS + warp; r < m;
-       r += static_cast<int64_t>(gridDim.x) * SWEEP_WARPS) {
-    float* wrow = Wp + r * n;
-    float w[4], s[4], z[4], ev[4];
-    unsigned qv[4];
+  const int rows_per_cta = SWEEP_WARPS * (32 / LPR);
+  for (int64_t rbase = static_cast<int64_t>(blockIdx.x) * rows_per_cta; rbase < m;
+       rbase += static_cast<int64_t>(gridDim.x) * rows_per_cta) {
+    const int64_t r = rbase + warp * (32 / LPR) + (lane / LPR);
+    const bool row_valid = r < m;
+    const int64_t rr = row_valid ? r : 0;  // inactive rows compute on row 0 and store nothing
+    float* wrow = Wp + rr * n;
+    float w[CPL], sc[CPL], zc[CPL], ev[CPL];
+    unsigned qv[CPL];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      w[c] = (4 * lane + c < bw) ? wrow[col0 + c] : 0.f;
-      s[c] = 1.f;
-      z[c] = 0.f;
-      ev[c] = 0.f;
-      qv[c] = 0u;
-      if (static_groups && 4 * lane + c < bw) {
-        const int g = perm[col0 + c] / G;
-        s[c] = scales[r * ng + g];
-        z[c] = zeros[r * ng + g];
+    for (int i = 0; i < CPL; i += 4) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (lane_valid) v = *reinterpret_cast<const float4*>(wrow + col0 + i);
+      w[i] = v.x;
+      w[i + 1] = v.y;
+      w[i + 2] = v.z;
+      w[i + 3] = v.w;
+    }
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      sc[i] = 1.f;
+      zc[i] = 0.f;
+      ev[i] = 0.f;
+      qv[i] = 0u;
+      if (static_groups && lane_valid) {
+        const int g = perm[col0 + i] / G;
+        sc[i] = scales[rr * ng + g];
+        zc[i] = zeros[rr * ng + g];
       }
     }
     if (!static_groups && !block_starts_group) {
-      // a group wider than the block started in an earlier block: its grid
-      // was written by that block's sweep
+      // a group wider than the block started in an earlier block
       const int64_t g = j1 / G;
-      const float gs = scales[r * ng + g], gz = zeros[r * ng + g];
+      const float gs = scales[rr * ng + g], gz = zeros[rr * ng + g];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        s[c] = gs;
-        z[c] = gz;
+      for (int i = 0; i < CPL; ++i) {
+        sc[i] = gs;
+        zc[i] = gz;
       }
     }
-    for (int j = 0; j < bw; ++j) {
-      if (!static_groups && (g_small ? ((j & (G - 1)) == 0) : (j == 0 && block_starts_group))) {
-        // group [j1 + j, j1 + j + G): min/max of its current values
-        float xmin = INFINITY, xmax = -INFINITY;
-        if (g_small) {
+    const int nchunks = bw / CPL;
+    for (int c = 0; c < nchunks; ++c) {
+      if (!SMALLG && !static_groups && (g_small ? (((c * CPL) & (G - 1)) == 0) : (c == 0 && block_starts_group)))
+        group_grid<SMALLG>(w, sc, zc, c * CPL, G, bw, q, g_small, wrow, j1, maxq, q == 0 && row_valid, scales,
+                           zeros, rr * ng);
+      const bool after = q > c;   // every column of this lane lies after the chunk
+      const bool own = q == c;    // this lane owns the chunk
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int k = 4 * lane + c;
-            if (k >= j && k < j + G && k < bw) {
-              xmin = fminf(xmin, w[c]);
-              xmax = fmaxf(xmax, w[c]);
-            }
-          }
-        } else {
-          // the group starts at this block and extends beyond it; every column
-          // of it is current (earlier blocks' updates are applied, this block's
-          // have not started)
-          for (int64_t k = j1 + lane; k < j1 + G; k += 32) {
-            const float v = wrow[k];
-            xmin = fminf(xmin, v);
-            xmax = fmaxf(xmax, v);
-          }
+      for (int jj = 0; jj < CPL; ++jj) {
+        const int j = c * CPL + jj;
+        if (SMALLG && !static_groups && ((j & (G - 1)) == 0))
+          group_grid<SMALLG>(w, sc, zc, j, G, bw, q, true, wrow, j1, maxq, q == 0 && row_valid, scales, zeros,
+                             rr * ng);
+        float e = 0.f;
+        if (own) {
+          // q = clip(rint(w / scale) + zero); w / scale is taken as w * (1 / scale),
+          // within an ulp of the quotient (the reciprocal is off the serial chain)
+          const float wj = w[jj], sj = sc[jj], zj = zc[jj];
+          const float rsj = 1.f / sj;
+          const float qq = fminf(fmaxf(rintf(wj * rsj) + zj, 0.f), maxq);
+          const float dq = sj * (qq - zj);
+          e = (wj - dq) * rU[j];
+          qv[jj] = static_cast<unsigned>(qq);
+          ev[jj] = e;
         }
-        for (int o = 16; o > 0; o >>= 1) {
-          xmin = fminf(xmin, __shfl_xor_sync(0xffffffffu, xmin, o));
-          xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, o));
-        }
-        float gs, gz;
-        grid_from_minmax(xmin, xmax, maxq, gs, gz);
+        e = __shfl_sync(0xffffffffu, e, c, LPR);
+        const float* urow = &Ub[upos(j, CPL * q)];  // 16 contiguous floats (one skew segment)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int k = 4 * lane + c;
-          if (!g_small || (k >= j && k < j + G)) {
-            s[c] = gs;
-            z[c] = gz;
+        for (int i = 0; i < CPL; i += 4) {
+          const float4 u = *reinterpret_cast<const float4*>(urow + i);
+          const float uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int t2 = 0; t2 < 4; ++t2) {
+            const bool act = after || (own && (i + t2 > jj));
+            const float upd = fmaf(-e, uu[t2], w[i + t2]);
+            w[i + t2] = act ? upd : w[i + t2];
           }
-        }
-        if (lane == 0) {
-          const int64_t g = (j1 + j) / G;
-          scales[r * ng + g] = gs;
-          zeros[r * ng + g] = gz;
         }
       }
-      const int owner = j >> 2, comp = j & 3;
-      const float4 u = *reinterpret_cast<const float4*>(&Ub[j * SB + 4 * lane]);
-      float e = 0.f;
-      if (lane == owner) {
-        float wj = w[0], sj = s[0], zj = z[0];
-#pragma unroll
-        for (int c = 1; c < 4; ++c)
-          if (comp == c) {
-            wj = w[c];
-            sj = s[c];
-            zj = z[c];
-          }
-        const float q = fminf(fmaxf(rintf(wj / sj) + zj, 0.f), maxq);
-        const float dq = sj * (q - zj);
-        e = (wj - dq) / Ub[j * SB + j];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (comp == c) {
-            qv[c] = static_cast<unsigned>(q);
-            ev[c] = e;
-          }
-      }
-      e = __shfl_sync(0xffffffffu, e, owner);
-      w[0] = fmaf(-e, u.x, w[0]);
-      w[1] = fmaf(-e, u.y, w[1]);
-      w[2] = fmaf(-e, u.z, w[2]);
-      w[3] = fmaf(-e, u.w, w[3]);
     }
-    if (4 * lane < bw) {
-      // bw is a multiple of 4 (n % 64 == 0), so a lane's 4 columns are all valid
-      const unsigned packed = qv[0] | (qv[1] << 8) | (qv[2] << 16) | (qv[3] << 24);
-      *reinterpret_cast<unsigned*>(codes8 + r * n + col0) = packed;
-      *reinterpret_cast<float4*>(Err + r * SB + 4 * lane) = make_float4(ev[0], ev[1], ev[2], ev[3]);
+    if (row_valid && lane_valid) {
+      uint4 pk;
+      pk.x = qv[0] | (qv[1] << 8) | (qv[2] << 16) | (qv[3] << 24);
+      pk.y = qv[4] | (qv[5] << 8) | (qv[6] << 16) | (qv[7] << 24);
+      pk.z = qv[8] | (qv[9] << 8) | (qv[10] << 16) | (qv[11] << 24);
+      pk.w = qv[12] | (qv[13] << 8) | (qv[14] << 16) | (qv[15] << 24);
+      *reinterpret_cast<uint4*>(codes8 + r * n + col0) = pk;
+#pragma unroll
+      for (int i = 0; i < CPL; i += 4)
+        *reinterpret_cast<float4*>(Err + r * SB + CPL * q + i) = make_float4(ev[i], ev[i + 1], ev[i + 2], ev[i + 3]);
     }
   }
 }
@@ -270,20 +334,26 @@ void launch_sweep_block(const Ctx& c, float* Wp, int64_t m, int64_t n, const flo
                         int wbits, bool static_groups, const int32_t* perm, float* scales, float* zeros,
                         unsigned char* codes8, float* Err) {
   static bool attr_done[64] = {false};
-  const int smem = SB * SB * 4;
+  const int smem = (SB * UPAD + SB) * 4;
   if (!attr_done[c.device & 63]) {
-    check_cuda(cudaFuncSetAttribute(sweep_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+    check_cuda(cudaFuncSetAttribute(sweep_block_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+               "cudaFuncSetAttribute(sweep)");
+    check_cuda(cudaFuncSetAttribute(sweep_block_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
                "cudaFuncSetAttribute(sweep)");
     attr_done[c.device & 63] = true;
   }
-  const int64_t rows_per_cta = SWEEP_WARPS;
+  const int64_t rows_per_cta = SWEEP_WARPS * 4;  // 4 rows per warp
   const int64_t want = (m + rows_per_cta - 1) / rows_per_cta;
-  const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(c.sm_count) * 3));
-  // (16 warps and 64 KB of shared memory per CTA: three CTAs per SM, so 4096
-  // rows run in a single wave)
-  sweep_block_kernel<<<grid, SWEEP_WARPS * 32, smem, c.stream>>>(
-      Wp, m, n, U, j1, G, static_cast<float>((1 << wbits) - 1), static_groups ? 1 : 0, perm, scales, zeros,
-      codes8, Err);
+  const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(c.sm_count) * 2));
+  const float maxq = static_cast<float>((1 << wbits) - 1);
+  const bool small_g = !static_groups && G < CPL;
+  if (small_g)
+    sweep_block_kernel<true><<<grid, SWEEP_WARPS * 32, smem, c.stream>>>(Wp, m, n, U, j1, G, maxq, static_groups ? 1 : 0,
+                                                                          perm, scales, zeros, codes8, Err);
+  else
+    sweep_block_kernel<false><<<grid, SWEEP_WARPS * 32, smem, c.stream>>>(Wp, m, n, U, j1, G, maxq,
+                                                                           static_groups ? 1 : 0, perm, scales, zeros,
+                                                                           codes8, Err);
   check_launch("sweep_block_kernel");
 }
 
