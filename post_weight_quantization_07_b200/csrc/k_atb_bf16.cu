@@ -303,7 +303,7 @@ __global__ void mirror_upper_kernel(float* H, int64_t n) {
 }  // namespace
 
 void launch_atb_bf16(const Ctx& c, const void* A, const void* B, int64_t n_tok, int64_t M,
-                     int64_t N, float alpha, float* C, int64_t ldc, bool upper_only) {
+                     int64_t N, float alpha, float* C, int64_t ldc, bool upper_only, int max_ctas) {
   if (n_tok <= 0 || M <= 0 || N <= 0) return;
   if ((M % 64) || (N % 64) || (ldc % 4)) fail(OC_ERR_INVALID_ARG, "atb_bf16: bad sizes");
   const CUtensorMap mA = make_tmap_2d(A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_tok, M, M, BK, 64, Swz::B128);
@@ -340,7 +340,8 @@ void launch_atb_bf16(const Ctx& c, const void* A, const void* B, int64_t n_tok, 
                "cudaFuncSetAttribute(atb_bf16)");
     attr_done[c.device & 63] = true;
   }
-  const int grid = static_cast<int>(std::min<int64_t>(p.units, c.sm_count));
+  const int ctas = (max_ctas > 0 && max_ctas < c.sm_count) ? max_ctas : c.sm_count;
+  const int grid = static_cast<int>(std::min<int64_t>(p.units, ctas));
   atb_bf16_kernel<<<grid, THREADS, SMEM_BYTES, c.stream>>>(mA, mB, mC, p);
   check_launch("atb_bf16_kernel");
 }

@@ -159,6 +159,17 @@ void check_launch(const char* kernel) {
   if (e != cudaSuccess) fail(OC_ERR_CUDA, "launch of %s failed: %s", kernel, cudaGetErrorString(e));
 }
 
+SideStream& side_stream(int device) {
+  static SideStream ss[64] = {};
+  SideStream& s = ss[device & 63];
+  if (s.stream == nullptr) {
+    check_cuda(cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking), "cudaStreamCreate(side)");
+    check_cuda(cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming), "cudaEventCreate(fork)");
+    check_cuda(cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming), "cudaEventCreate(join)");
+  }
+  return s;
+}
+
 CUtensorMap make_tmap_2d(const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t rows, uint64_t cols,
                          uint64_t ld, uint32_t box_rows, uint32_t box_cols, Swz swz) {
   if (!aligned16(base)) fail(OC_ERR_INVALID_ARG, "TMA base address must be 16-byte aligned");
@@ -487,8 +498,9 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
     sizing.take<float>(nn);                 // d -> M -> U
     sizing.take<float>(nn);                 // d^T hi -> inverse factor -> U hi
     sizing.take<float>(nn + 4096);          // d^T lo -> recursion scratch -> U lo
-    sizing.take<float>(nn);                 // U^T hi
-    sizing.take<float>(nn);                 // U^T lo
+    sizing.take<float>(nn);                 // factor input -> U -> U^T hi
+    sizing.take<float>(nn);                 // inverse factor -> U^T lo
+    sizing.take<float>(nn + 4096);          // factor recursion scratch
     sizing.take<float>(mn);                 // hi halves (W, G, T)
     sizing.take<float>(mn);                 // lo halves
     sizing.take<float>(mn);                 // G -> T
@@ -505,6 +517,7 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
     float* scratch = cv.take<float>(nn + 4096);
     float* UTh = cv.take<float>(nn);
     float* UTl = cv.take<float>(nn);
+    float* Fs = cv.take<float>(nn + 4096);
     float* Ph = cv.take<float>(mn);
     float* Pl = cv.take<float>(mn);
     float* G2 = cv.take<float>(mn);
@@ -524,10 +537,35 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
       launch_atb_bf16(c, Xhat, Xhat, n_tok, n, n, 2.0f, H, n, true);
       launch_mirror_upper(c, H, n);
     }
+    // GPTQ's dampened Hessian equals QEP's 2A unless a column is dead (their
+    // dampening constants then differ): one device-to-host read decides.
+    launch_diag_stats(c, H, n, damp, 1.0f, true, stats, dead);
+    DiagStats hs{};
+    check_cuda(cudaMemcpyAsync(&hs, stats, sizeof(DiagStats), cudaMemcpyDeviceToHost, c.stream), "read stats");
+    check_cuda(cudaStreamSynchronize(c.stream), "cudaStreamSynchronize");
+    if (hs.nonfinite) return finish(c);
+    // The factorisation needs only H.  With no dead column (one factorisation
+    // serves QEP and GPTQ) it runs on a side stream, on a few SMs, while the
+    // cross product X^T Xhat occupies the rest; it factors into UTh (input
+    // reversed and dampened, output U) with UTl and Fs as its scratch.
+    const bool shared_factor = hs.n_dead == 0;
+    SideStream& ss = side_stream(c.device);
+    Ctx cs = c;
+    cs.stream = ss.stream;
+    if (shared_factor) {
+      check_cuda(cudaEventRecord(ss.fork, c.stream), "cudaEventRecord(fork)");
+      check_cuda(cudaStreamWaitEvent(cs.stream, ss.fork, 0), "cudaStreamWaitEvent(fork)");
+      PhaseScope ps(cs, kPhFactor);
+      if (act_order) launch_act_order_perm(cs, H, n, perm);
+      else launch_identity_perm(cs, n, perm);
+      launch_build_reversed(cs, H, n, perm, stats, 1.0f, true, UTh);
+      factor_inverse_upper(cs, UTh, UTl, Fs, UTh, n, true, fsplit);
+      check_cuda(cudaEventRecord(ss.join, cs.stream), "cudaEventRecord(join)");
+    }
     {
       PhaseScope ps(c, kPhQepCross);
       check_cuda(cudaMemsetAsync(D, 0, nn * sizeof(float), c.stream), "memset d");
-      launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false);
+      launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false, shared_factor ? c.sm_count - kSideSMs : 0);
       launch_sub_half(c, D, H, n);
     }
     {
@@ -536,14 +574,7 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
       split_tf32(c, W, m, n, n, Ph, Pl, n);
       gemm_tf32x3(c, m, n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, G2, n, kANone);
     }
-    // GPTQ's dampened Hessian equals QEP's 2A unless a column is dead (their
-    // dampening constants then differ): one device-to-host read decides.
-    launch_diag_stats(c, H, n, damp, 1.0f, true, stats, dead);
-    DiagStats hs{};
-    check_cuda(cudaMemcpyAsync(&hs, stats, sizeof(DiagStats), cudaMemcpyDeviceToHost, c.stream), "read stats");
-    check_cuda(cudaStreamSynchronize(c.stream), "cudaStreamSynchronize");
-    if (hs.nonfinite) return finish(c);
-    if (hs.n_dead > 0) {
+    if (!shared_factor) {
       // two factorisations: QEP's own (original order), then GPTQ's
       {
         PhaseScope ps(c, kPhFactor);
@@ -577,17 +608,11 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
         if (act_order) launch_static_grid(c, W_out, m, n, static_cast<int>(G), wbits, dead, scales, zeros);
       }
     } else {
-      // one factorisation of P H_d P^T; QEP applied in processing order:
-      //   W'P = WP + 2 alpha ((G P) U^T) U
-      {
-        PhaseScope ps(c, kPhFactor);
-        if (act_order) launch_act_order_perm(c, H, n, perm);
-        else launch_identity_perm(c, n, perm);
-        launch_build_reversed(c, H, n, perm, stats, 1.0f, true, D);
-        factor_inverse_upper(c, D, Xi, scratch, D, n, true, fsplit);
-      }
+      check_cuda(cudaStreamWaitEvent(c.stream, ss.join, 0), "cudaStreamWaitEvent(join)");
+      // QEP applied in processing order: W'P = WP + 2 alpha ((G P) U^T) U
       {
         PhaseScope ps(c, kPhQepApply);
+        check_cuda(cudaMemcpyAsync(D, UTh, nn * sizeof(float), cudaMemcpyDeviceToDevice, c.stream), "copy U");
         const float* U = D;
         split_tf32(c, U, n, n, n, Xi, scratch, n);
         split_tf32(c, U, n, n, n, UTh, UTl, n, true);

@@ -93,8 +93,19 @@ CUtensorMap make_tmap_2d(const void* base, CUtensorMapDataType dt, int elem_byte
 // C[i][j] += alpha * sum_t A[t][i] * B[t][j] with A, B bf16 token-major
 // [n_tok x M] and [n_tok x N]; C fp32 [M x N] (ldc).  upper_only: A == B and
 // only tiles touching the upper triangle are computed (the caller mirrors).
+// max_ctas > 0 caps the persistent grid (leaving SMs free for concurrent work).
 void launch_atb_bf16(const Ctx& c, const void* A, const void* B, int64_t n_tok, int64_t M,
-                     int64_t N, float alpha, float* C, int64_t ldc, bool upper_only);
+                     int64_t N, float alpha, float* C, int64_t ldc, bool upper_only, int max_ctas = 0);
+
+// Per-device side stream and fork/join events for running the (latency
+// bound) factorisation beside a tensor-core product on the call's stream.
+struct SideStream {
+  cudaStream_t stream;
+  cudaEvent_t fork, join;
+};
+SideStream& side_stream(int device);
+// SMs left to the side stream while the main stream's product runs.
+constexpr int kSideSMs = 8;
 
 // Mirror the upper triangle of an n x n matrix into its lower triangle.
 void launch_mirror_upper(const Ctx& c, float* H, int64_t n);
