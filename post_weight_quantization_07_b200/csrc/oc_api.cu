@@ -322,6 +322,9 @@ int oc_hessian_accumulate(const void* X, int64_t n_tok, int64_t n, float* H, voi
     {
       PhaseScope ps(c, kPhHessian);
       launch_atb_bf16(c, X, X, n_tok, n, n, 2.0f, H, n, true);
+    }
+    {
+      PhaseScope ps(c, kPhHessianFix);
       launch_mirror_upper(c, H, n);
     }
     return finish(c);
@@ -381,9 +384,15 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
       Hp = Hs;
     }
     {
-      PhaseScope ps(c, kPhQepCross);
+      PhaseScope ps(c, kPhQepCrossFix);
       check_cuda(cudaMemsetAsync(D, 0, nn * sizeof(float), c.stream), "memset D");
+    }
+    {
+      PhaseScope ps(c, kPhQepCross);
       launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false);
+    }
+    {
+      PhaseScope ps(c, kPhQepCrossFix);
       launch_sub_half(c, D, Hp, n);
     }
     {
@@ -532,9 +541,15 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
     DiagStats* stats = cv.take<DiagStats>(1);
 
     {
-      PhaseScope ps(c, kPhHessian);
+      PhaseScope ps(c, kPhHessianFix);
       check_cuda(cudaMemsetAsync(H, 0, nn * sizeof(float), c.stream), "memset H");
+    }
+    {
+      PhaseScope ps(c, kPhHessian);
       launch_atb_bf16(c, Xhat, Xhat, n_tok, n, n, 2.0f, H, n, true);
+    }
+    {
+      PhaseScope ps(c, kPhHessianFix);
       launch_mirror_upper(c, H, n);
     }
     // GPTQ's dampened Hessian equals QEP's 2A unless a column is dead (their
@@ -563,9 +578,15 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
       check_cuda(cudaEventRecord(ss.join, cs.stream), "cudaEventRecord(join)");
     }
     {
-      PhaseScope ps(c, kPhQepCross);
+      PhaseScope ps(c, kPhQepCrossFix);
       check_cuda(cudaMemsetAsync(D, 0, nn * sizeof(float), c.stream), "memset d");
+    }
+    {
+      PhaseScope ps(c, kPhQepCross);
       launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false, shared_factor ? c.sm_count - kSideSMs : 0);
+    }
+    {
+      PhaseScope ps(c, kPhQepCrossFix);
       launch_sub_half(c, D, H, n);
     }
     {

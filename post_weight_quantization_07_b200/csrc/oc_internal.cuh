@@ -44,8 +44,8 @@ void check_launch(const char* kernel);
 
 // ------------------------------------------------------------------ profiling
 enum Phase : int {
-  kPhHessian = 0,   // oc_hessian_accumulate: tensor-core SYRK + mirror
-  kPhQepCross,      // X^T Xhat on the tensor cores, minus Xhat^T Xhat
+  kPhHessian = 0,   // the tensor-core SYRK launch of the Hessian (one launch)
+  kPhQepCross,      // the tensor-core X^T Xhat launch (one launch)
   kPhQepSyrk,       // Xhat^T Xhat when no H is supplied
   kPhQepWDelta,     // G = W d
   kPhFactor,        // dampening, reversal, blocked Cholesky + inverse, reversal
@@ -54,6 +54,8 @@ enum Phase : int {
   kPhGptqSweep,     // 128-column block sweeps
   kPhGptqTrailing,  // trailing updates of later columns
   kPhGptqPack,      // inverse permutation + bit packing
+  kPhHessianFix,    // clearing H, mirroring its upper triangle
+  kPhQepCrossFix,   // clearing d, subtracting Xhat^T Xhat
   kNumPhases
 };
 

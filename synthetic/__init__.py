@@ -137,9 +137,14 @@ def _base_std(spec: LayerSpec) -> float:
 def bf16_round(a: np.ndarray) -> np.ndarray:
     """Round float32/float64 values to the nearest bf16 (ties to even), returned as float32."""
     a32 = np.ascontiguousarray(a, dtype=np.float32)
-    u = a32.view(np.uint32).astype(np.uint64)
-    rounded = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    out = rounded.astype(np.uint32).view(np.float32)
+    u = a32.view(np.uint32)
+    # For finite inputs the sum stays below 2^32 (the largest finite pattern is
+    # 0xFF7FFFFF), so 32-bit arithmetic cannot wrap.
+    rounded = (u >> 16) & np.uint32(1)
+    rounded += u
+    rounded += np.uint32(0x7FFF)
+    rounded &= np.uint32(0xFFFF0000)
+    out = rounded.view(np.float32)
     # NaN/Inf are not produced by these recipes; keep them untouched if present.
     bad = ~np.isfinite(a32)
     if bad.any():
