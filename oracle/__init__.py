@@ -96,7 +96,7 @@ def qep_cross(x, xhat, chunk: int = 8192):
     return d
 
 
-def qep_correct(W, x, xhat, alpha: float, damp: float, H=None, chunk: int = 8192):
+def qep_correct(W, x, xhat, alpha: float, damp: float, H=None, chunk: int = 8192, d=None):
     """QEP weight correction [OneComp-release, section "量化錯誤傳播 (QEP)"].
 
     The corrected weight makes the quantised layer, fed the perturbed inputs Xh,
@@ -105,11 +105,13 @@ def qep_correct(W, x, xhat, alpha: float, damp: float, H=None, chunk: int = 8192
         W* = W + W d A^-1,  d = (X - Xh)^T Xh,  A = Xh^T Xh + lam I,
     and QEP moves a fraction alpha of the way: W' = W + alpha * W d A^-1, with
     lam = damp * mean(diag(Xh^T Xh)).  If H (= 2 Xh^T Xh over the same tokens)
-    is given it replaces the recomputation of Xh^T Xh.
+    is given it replaces the recomputation of Xh^T Xh; likewise d (= the
+    qep_cross of the same tokens) replaces the recomputation of the cross
+    term, and x, xhat are then not read.
     """
     W = _f64(W)
     S = hessian(xhat, chunk=chunk) / 2.0 if H is None else _f64(H) / 2.0
-    d = qep_cross(x, xhat, chunk=chunk)
+    d = qep_cross(x, xhat, chunk=chunk) if d is None else _f64(d)
     n = S.shape[0]
     lam = damp * float(np.mean(np.diag(S)))
     A = S + lam * np.eye(n)

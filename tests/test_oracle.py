@@ -364,3 +364,17 @@ def test_workload_recipes_shapes():
     assert CONFIGS["c2_q_proj"].outlier_count() == 40
     assert CONFIGS["c3_down_proj"].outlier_count() == 55
     assert CONFIGS["c5_70b_down"].outlier_count() == 286
+
+
+def test_qep_precomputed_terms_over_chunks():
+    # H and d are sums over tokens: accumulating them over token chunks and
+    # passing them in must give the same W' as the one-shot computation.
+    rng = np.random.default_rng(71)
+    x = rng.standard_normal((300, 16))
+    xh = x + 0.1 * rng.standard_normal(x.shape)
+    W = rng.standard_normal((5, 16))
+    H = sum(oracle.hessian(xh[t:t + 64]) for t in range(0, 300, 64))
+    d = sum(oracle.qep_cross(x[t:t + 64], xh[t:t + 64]) for t in range(0, 300, 64))
+    a = oracle.qep_correct(W, x, xh, 0.5, 0.01)
+    b = oracle.qep_correct(W, None, None, 0.5, 0.01, H=H, d=d)
+    assert np.allclose(a, b, rtol=0, atol=1e-12)
