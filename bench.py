@@ -35,6 +35,7 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 SM_COUNT = 148
+L2_BYTES = 126 * 1024 * 1024
 CPU_SAMPLE_TOKENS = 16384
 CPU_SAMPLE_ROWS = 2048
 # DRAM bytes (read + written) per launch of atb_bf16_kernel, the mean of its
@@ -53,16 +54,31 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+WORKLOAD_TITLES = {
+    "c1_512": "single 512x512 linear layer",
+    "c2_q_proj": "Llama-2-7B q_proj layer",
+    "c3_down_proj": "Llama-2-7B MLP down_proj layer",
+    "c5_70b_down": "Llama-3-70B-shaped MLP down_proj layer",
+}
+X_KINDS = {"normal": "N(0,1)", "t": "Student-t({nu:g})", "swiglu": "SiLU(z1)*z2"}
+
+
 def workload_config(spec):
+    xk = X_KINDS.get(spec.x_kind, spec.x_kind).format(nu=spec.nu)
+    outl = f"{spec.outlier_count()} channels x{spec.outlier_scale:g}"
+    noise = (f"Xhat = X + N(0, {spec.noise_abs:g}^2)" if spec.noise_abs > 0
+             else f"Xhat = X + {100 * spec.noise_rel:g}% channel noise")
+    x_bytes = spec.n_tok * spec.d_in * 2
     return {
-        "workload": (f"{spec.name}: Llama-2-7B q_proj layer {spec.d_out}x{spec.d_in}, "
-                     f"{spec.n_tok} calibration tokens (bf16 Student-t(4), 1% channels x20, "
-                     f"Xhat = X + 2% channel noise), QEP alpha {spec.alpha}, GPTQ "
-                     f"{spec.wbits}-bit g{spec.groupsize} asymmetric, damp {spec.damp}, "
+        "workload": (f"{spec.name}: {WORKLOAD_TITLES.get(spec.name, 'linear layer')} "
+                     f"{spec.d_out}x{spec.d_in}, {spec.n_tok} calibration tokens (bf16 {xk}, "
+                     f"{outl}, {noise}), QEP alpha {spec.alpha}, GPTQ {spec.wbits}-bit "
+                     f"g{spec.groupsize} asymmetric, damp {spec.damp}, "
                      f"act_order {'on' if spec.act_order else 'off'}"),
         "d_out": spec.d_out, "d_in": spec.d_in, "n_tok": spec.n_tok, "wbits": spec.wbits,
         "groupsize": spec.groupsize, "act_order": spec.act_order,
-        "l2": "inputs larger than L2 (X and Xhat are 2.1 GB each), no flush needed",
+        "l2": (f"inputs larger than L2 (X and Xhat are {x_bytes / 1e9:.2f} GB each), no flush needed"
+               if x_bytes > L2_BYTES else "inputs fit in L2: L2 flushed between steps"),
     }
 
 
@@ -355,11 +371,26 @@ def run_ours(args, rank, world, local_rank):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     props = torch.cuda.get_device_properties(local_rank)
     bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+    # Inputs smaller than L2 would be re-read from cache: then every step is
+    # timed alone, after a write of a buffer larger than L2 outside its events.
+    fits_l2 = X.numel() * X.element_size() <= L2_BYTES
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if fits_l2 else None
+    step_ms = 0.0
     with ClockSampler(gpu_index_for(local_rank), bus) as clk:
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
+        if fits_l2:
+            for _ in range(args.steps):
+                flush.fill_(1.0)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                step()
+                b.record(stream)
+                b.synchronize()
+                step_ms += a.elapsed_time(b)
+        else:
+            e0.record(stream)
+            for _ in range(args.steps):
+                step()
+            e1.record(stream)
         barrier()
     launches = oc.oc_launch_count() - launches0
     oc.oc_profile_enable(False)
@@ -367,7 +398,7 @@ def run_ours(args, rank, world, local_rank):
     st = oc.oc_stream_status(stream)
     if st != oc.OC_OK:
         raise RuntimeError(f"timed steps failed: {oc.oc_status_string(st)}")
-    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_total = max_over_ranks(step_ms if fits_l2 else e0.elapsed_time(e1))
     ms_per_step = ms_total / args.steps
     value = world * args.steps / (ms_total / 1e3)
 

@@ -176,8 +176,11 @@ def inv_chol_upper_reversed(Hd):
     n = Hd.shape[0]
     rev = np.arange(n)[::-1]
     L = np.linalg.cholesky(Hd[np.ix_(rev, rev)])
-    Linv = sla.solve_triangular(L, np.eye(n), lower=True)
-    return Linv[np.ix_(rev, rev)]
+    # triangular inverse (LAPACK trtri): L^-1, lower
+    Linv, info = sla.lapack.dtrtri(L, lower=1)
+    if info != 0:
+        raise np.linalg.LinAlgError(f"trtri failed ({info})")
+    return np.tril(Linv)[np.ix_(rev, rev)]
 
 
 # ----------------------------------------------------------------------------- grid
@@ -304,21 +307,23 @@ def gptq_sweep(Wp, U, wbits: int, groupsize: int, perm=None, static=None, block:
 
 
 def gptq_quantize(W, H, wbits: int, groupsize: int, damp: float, act_order: bool,
-                  block: int = 256, unblocked: bool = False, perm=None):
+                  block: int = 256, unblocked: bool = False, perm=None, U=None):
     """GPTQ with per-group asymmetric grid, returning outputs in original order.
 
     Returns dict(codes = m x n int codes in original column order, packed = the
     uint32 bitstream, scales, zeros = m x (n/G), deq = dequantised weights in
     original order, perm = processing order, U = the inverse-Hessian factor).
     ``perm`` overrides the act_order order (used to replay another
-    implementation's tie-breaking).
+    implementation's tie-breaking).  ``U``, if given, is the factor of this
+    same preparation (inv_chol_upper of its Hd, e.g. from an earlier call on
+    other rows of W) and is used instead of recomputing it.
     """
     prep = gptq_prepare(W, H, damp, act_order, perm=perm)
     perm = prep["perm"]
     n = perm.shape[0]
     maxq = (1 << wbits) - 1
     G = _group_size(groupsize, n)
-    U = inv_chol_upper(prep["Hd"])
+    U = inv_chol_upper(prep["Hd"]) if U is None else _f64(U)
     static = None
     if act_order:
         Wd = prep["W_dead"]
@@ -406,7 +411,7 @@ def _half_dist(v):
 
 def teacher_forced_check(W, H, wbits: int, groupsize: int, damp: float, act_order: bool,
                          codes, scales, zeros, perm=None, rows=None, block: int = 256,
-                         boundary_tol: float = 1e-3):
+                         boundary_tol: float = 1e-3, U=None):
     """Replay the sweep with another implementation's decisions forced in.
 
     Runs the float64 sweep row by row, but for every column uses the candidate's
@@ -416,7 +421,8 @@ def teacher_forced_check(W, H, wbits: int, groupsize: int, damp: float, act_orde
     v = w/scale, it measures v's distance to the nearest half-integer.  Returns
     counts and the worst distances; the candidate passes when every mismatch is
     a single step within ``boundary_tol`` of a boundary and every scale is within
-    the caller's tolerance of the oracle's.
+    the caller's tolerance of the oracle's.  ``U``, if given, is the factor of
+    this same preparation (as in gptq_quantize).
     """
     codes = np.asarray(codes)
     scales = _f64(scales)
@@ -430,7 +436,7 @@ def teacher_forced_check(W, H, wbits: int, groupsize: int, damp: float, act_orde
     G = _group_size(groupsize, n)
     prep = gptq_prepare(W, H, damp, act_order, perm=perm)
     perm = prep["perm"]
-    U = inv_chol_upper(prep["Hd"])
+    U = inv_chol_upper(prep["Hd"]) if U is None else _f64(U)
     codes_p = codes[:, perm]
     stats = {"n_codes": m * n, "n_mismatch": 0, "n_bad": 0, "max_mismatch_dist": 0.0,
              "scale_max_rel": 0.0, "zero_mismatch": 0, "zero_bad": 0}

@@ -378,3 +378,20 @@ def test_qep_precomputed_terms_over_chunks():
     a = oracle.qep_correct(W, x, xh, 0.5, 0.01)
     b = oracle.qep_correct(W, None, None, 0.5, 0.01, H=H, d=d)
     assert np.allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_gptq_given_factor_equals_recomputed():
+    # Passing the factor of the same preparation (here by the reversed route,
+    # which is pinned equal to route A) must not change any output.
+    rng = np.random.default_rng(72)
+    X = rng.standard_normal((200, 64))
+    H = oracle.hessian(X)
+    W = rng.standard_normal((6, 64))
+    a = oracle.gptq_quantize(W, H, 3, 16, 0.01, True)
+    prep = oracle.gptq_prepare(W, H, 0.01, True)
+    U = oracle.inv_chol_upper_reversed(prep["Hd"])
+    b = oracle.gptq_quantize(W, H, 3, 16, 0.01, True, U=U)
+    assert np.array_equal(a["codes"], b["codes"])
+    assert np.allclose(a["scales"], b["scales"], rtol=1e-12, atol=0)
+    st = oracle.teacher_forced_check(W, H, 3, 16, 0.01, True, a["codes"], a["scales"], a["zeros"], U=U)
+    assert st["n_mismatch"] == 0 and st["scale_max_rel"] <= 1e-12
