@@ -151,6 +151,8 @@ constexpr int LDA = LEAF + 1;      // padded leading dimensions (bank spread)
 constexpr int LDT = LEAF / 2 + 1;
 
 struct LeafSmem {
+  float4 col4[32];                 // 4 columns of the current 32 block, one row per lane
+  float4 blk[4];                   // the current 4x4 pivot block
   float A[LEAF * LDA];
   float X[LEAF * LDA];
   float T[(LEAF / 2) * LDT];       // L21 of the 128 level; temporaries of the 64 level
@@ -159,25 +161,55 @@ struct LeafSmem {
   float R32[32];                   // reciprocals of its diagonal
 };
 
-__device__ __forceinline__ void warp_chol_inv32(LeafSmem& sm, int off, int* status) {
+// One step of the 32x32 factor: columns K..K+3.  The 4x4 pivot block is
+// factored redundantly by every lane in registers; each lane then finishes its
+// own row's four entries, and the four columns reach the other lanes as one
+// float4 per row through shared memory.
+template <int K>
+__device__ __forceinline__ void chol32_step(LeafSmem& sm, float (&a)[32], int lane, bool& bad) {
+  if (lane >= K && lane < K + 4) sm.blk[lane - K] = make_float4(a[K], a[K + 1], a[K + 2], a[K + 3]);
+  __syncwarp();
+  const float4 q0 = sm.blk[0], q1 = sm.blk[1], q2 = sm.blk[2], q3 = sm.blk[3];
+  const float r0 = rsqrtf(q0.x);
+  const float l10 = q1.x * r0, l20 = q2.x * r0, l30 = q3.x * r0;
+  const float d1 = fmaf(-l10, l10, q1.y);
+  const float r1 = rsqrtf(d1);
+  const float l21 = fmaf(-l20, l10, q2.y) * r1, l31 = fmaf(-l30, l10, q3.y) * r1;
+  const float d2 = fmaf(-l21, l21, fmaf(-l20, l20, q2.z));
+  const float r2 = rsqrtf(d2);
+  const float l32 = fmaf(-l31, l21, fmaf(-l30, l20, q3.z)) * r2;
+  const float d3 = fmaf(-l32, l32, fmaf(-l31, l31, fmaf(-l30, l30, q3.w)));
+  const float r3 = rsqrtf(d3);
+  if (!(q0.x > 0.f) || !(d1 > 0.f) || !(d2 > 0.f) || !(d3 > 0.f) || !isfinite(q0.x + d1 + d2 + d3)) bad = true;
+  const float x0 = a[K] * r0;
+  const float x1 = fmaf(-x0, l10, a[K + 1]) * r1;
+  const float x2 = fmaf(-x1, l21, fmaf(-x0, l20, a[K + 2])) * r2;
+  const float x3 = fmaf(-x2, l32, fmaf(-x1, l31, fmaf(-x0, l30, a[K + 3]))) * r3;
+  const int rr = lane - K;  // rows of the pivot block keep zeros above the diagonal
+  a[K] = x0;
+  a[K + 1] = (rr >= 0 && rr < 1) ? 0.f : x1;
+  a[K + 2] = (rr >= 0 && rr < 2) ? 0.f : x2;
+  a[K + 3] = (rr >= 0 && rr < 3) ? 0.f : x3;
+  if constexpr (K + 4 < 32) {
+    sm.col4[lane] = make_float4(a[K], a[K + 1], a[K + 2], a[K + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int j = K + 4; j < 32; ++j) {
+      const float4 v = sm.col4[j];
+      if (lane >= j)
+        a[j] = fmaf(-a[K + 3], v.w, fmaf(-a[K + 2], v.z, fmaf(-a[K + 1], v.y, fmaf(-a[K], v.x, a[j]))));
+    }
+    chol32_step<K + 4>(sm, a, lane, bad);
+  }
+}
+
+__device__ __noinline__ void warp_chol_inv32(LeafSmem& sm, int off, int* status) {
   const int lane = threadIdx.x & 31;
   float a[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) a[j] = (j <= lane) ? sm.A[(off + lane) * LDA + off + j] : 0.f;
   bool bad = false;
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    const float d = __shfl_sync(0xffffffffu, a[k], k);
-    if (!(d > 0.f) || !isfinite(d)) bad = true;
-    const float rsd = rsqrtf(d);
-    const float lk = a[k] * rsd;  // L[lane][k] (0 above the diagonal)
-    a[k] = lk;
-#pragma unroll
-    for (int j = k + 1; j < 32; ++j) {
-      const float ljk = __shfl_sync(0xffffffffu, lk, j);
-      if (lane >= j) a[j] = fmaf(-lk, ljk, a[j]);
-    }
-  }
+  chol32_step<0>(sm, a, lane, bad);
   if (bad && lane == 0) record_error(status, kDevNotSpd);
   float dl = 1.f;
 #pragma unroll

@@ -163,7 +163,11 @@ SideStream& side_stream(int device) {
   static SideStream ss[64] = {};
   SideStream& s = ss[device & 63];
   if (s.stream == nullptr) {
-    check_cuda(cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking), "cudaStreamCreate(side)");
+    // Highest priority: when SMs free up, the factorisation's kernels are
+    // placed before the next piece of the cross product.
+    int least = 0, greatest = 0;
+    check_cuda(cudaDeviceGetStreamPriorityRange(&least, &greatest), "cudaDeviceGetStreamPriorityRange");
+    check_cuda(cudaStreamCreateWithPriority(&s.stream, cudaStreamNonBlocking, greatest), "cudaStreamCreate(side)");
     check_cuda(cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming), "cudaEventCreate(fork)");
     check_cuda(cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming), "cudaEventCreate(join)");
   }
@@ -583,7 +587,21 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
     }
     {
       PhaseScope ps(c, kPhQepCross);
-      launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false, shared_factor ? c.sm_count - kSideSMs : 0);
+      if (shared_factor) {
+        // In token ranges: between two launches the high-priority factorisation
+        // can take the freed SMs for its wide tensor-core products.
+        const int64_t parts = std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens));
+        const int64_t per = ((n_tok + parts - 1) / parts + 63) / 64 * 64;
+        const unsigned char* xb = static_cast<const unsigned char*>(X);
+        const unsigned char* hb = static_cast<const unsigned char*>(Xhat);
+        for (int64_t t0 = 0; t0 < n_tok; t0 += per) {
+          const int64_t len = std::min(per, n_tok - t0);
+          launch_atb_bf16(c, xb + t0 * n * 2, hb + t0 * n * 2, len, n, n, 1.0f, D, n, false,
+                          c.sm_count - kSideSMs);
+        }
+      } else {
+        launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false, 0);
+      }
     }
     {
       PhaseScope ps(c, kPhQepCrossFix);

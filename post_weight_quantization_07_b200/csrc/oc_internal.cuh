@@ -108,6 +108,10 @@ struct SideStream {
 SideStream& side_stream(int device);
 // SMs left to the side stream while the main stream's product runs.
 constexpr int kSideSMs = 8;
+// The cross product beside it runs as up to kCrossParts launches over token
+// ranges of at least kCrossPartMinTokens tokens each.
+constexpr int64_t kCrossParts = 32;
+constexpr int64_t kCrossPartMinTokens = 8192;
 
 // Mirror the upper triangle of an n x n matrix into its lower triangle.
 void launch_mirror_upper(const Ctx& c, float* H, int64_t n);
