@@ -536,6 +536,88 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- one 7B block
+
+BLOCK_GROUPS = ((0, 1, 2), (3,), (4, 5), (6,))  # q/k/v, o, gate/up, down of llama7b_layers()
+
+
+def run_block(args, rank, world, local_rank):
+    """One Llama-2-7B-shaped transformer block: q/k/v quantised as one group on
+    their shared input, o alone, gate/up as one group, down alone (7 layers,
+    4 calls).  Each group's X, Xhat follow its first layer's recipe; every
+    layer has its own seeded W ~ N(0, 0.02^2) rounded to bf16."""
+    import torch
+
+    import post_weight_quantization_07_b200 as oc
+    from synthetic import llama7b_layers, make_layer_device
+
+    torch.cuda.set_device(local_rank)
+    n_tok = args.n_tok or 131072
+    specs = llama7b_layers(n_tok)[:7]
+    groups = []
+    for g in BLOCK_GROUPS:
+        lead = specs[g[0]]
+        L = make_layer_device(lead.with_(seed=lead.seed + 1000 * rank), "cuda")
+        Ws = []
+        for j in g:
+            gen = torch.Generator(device="cuda").manual_seed(specs[j].seed + 1000 * rank)
+            w = torch.randn(specs[j].d_out, specs[j].d_in, generator=gen, device="cuda") * specs[j].w_std
+            Ws.append(w.to(torch.bfloat16).float().contiguous())
+        groups.append((lead, Ws, L["X"], L["Xhat"]))
+        del L
+    stream = torch.cuda.current_stream()
+    oc.oc_set_sync(False)
+    outs = []
+    for lead, Ws, X, Xh in groups:
+        n = lead.d_in
+        G = lead.groupsize
+        outs.append(dict(H=torch.empty(n, n, device="cuda"), W_outs=[torch.empty_like(w) for w in Ws],
+                         codes=[torch.empty(w.shape[0], n * lead.wbits // 32, dtype=torch.int32, device="cuda")
+                                for w in Ws],
+                         scales=[torch.empty(w.shape[0], n // G, device="cuda") for w in Ws],
+                         zeros=[torch.empty(w.shape[0], n // G, device="cuda") for w in Ws]))
+
+    def step():
+        for (lead, Ws, X, Xh), o in zip(groups, outs):
+            oc.oc_quantize_layer_group(Ws, X, Xh, lead.alpha, lead.damp, lead.wbits, lead.groupsize,
+                                       lead.act_order, stream=stream, **o)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    launches0 = oc.oc_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(local_rank)
+    bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+    with ClockSampler(gpu_index_for(local_rank), bus) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    st = oc.oc_stream_status(stream)
+    if st != oc.OC_OK:
+        raise RuntimeError(f"block steps failed: {oc.oc_status_string(st)}")
+    ms_block = e0.elapsed_time(e1) / args.steps
+    layers = sum(len(g) for g in BLOCK_GROUPS)
+    line = {
+        "metric": METRIC, "value": round(layers / (ms_block / 1e3), 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_block, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16+f32",
+        "data": "synthetic",
+        "config": {"workload": (f"c4_block: one Llama-2-7B-shaped block (q/k/v/o 4096x4096 4-bit, gate/up "
+                                f"4096->11008 and down 11008->4096 3-bit, g128, QEP alpha 0.5, damp 0.01), "
+                                f"{n_tok} calibration tokens per input, q/k/v and gate/up sharing their "
+                                f"inputs (one Hessian, cross term and factorisation per group)"),
+                   "layers_per_step": layers, "calls_per_step": len(BLOCK_GROUPS),
+                   "l2": "inputs larger than L2, no flush needed"},
+        "seconds_per_32_block_model": round(32 * ms_block / 1e3, 3),
+        "gpu_launches": int(oc.oc_launch_count() - launches0), "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
@@ -589,6 +671,8 @@ def main():
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.workload == "c4_block":
+        run_block(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

@@ -204,6 +204,30 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
                       float* zeros, int32_t* perm_out, void* stream);
 
 /*
+ * Several layers that read the same calibration inputs, e.g. the q, k and v
+ * projections of one attention block or gate and up of one MLP (the One
+ * Compression hub page, section "核心功能拆解", quantises a model layer by
+ * layer; layers fed the same activations have the same Hessian).  For each
+ * layer l the results are those of oc_quantize_layer(W[l], m[l], ...) with
+ * the shared n, X, Xhat and settings; H, the cross term d and the
+ * inverse-Hessian factor depend only on the inputs and are computed once.
+ *   count     1..16 layers.
+ *   W, W_out, codes, scales, zeros: host arrays of `count` device pointers,
+ *             each as in oc_quantize_layer for a layer of m[l] rows
+ *             (m: host array of `count` row counts).  No W_out[l] may alias
+ *             any W[k].
+ *   H         fp32 [n x n], written once.   perm_out: the shared processing
+ *             order (optional).
+ * Errors are those of oc_quantize_layer; a bad argument of any layer fails
+ * the call before any launch.
+ */
+int oc_quantize_layer_group(int count, const float* const* W, const int64_t* m, int64_t n,
+                            const void* X, const void* Xhat, int64_t n_tok, float alpha, float damp,
+                            int wbits, int groupsize, int act_order, float* H,
+                            float* const* W_out, uint32_t* const* codes, float* const* scales,
+                            float* const* zeros, int32_t* perm_out, void* stream);
+
+/*
  * Allocation-free GPTQ (no counterpart in the paper: an addition for callers of
  * this library).  Some callers cannot have a library allocate device memory on
  * its own -- e.g. a process whose memory is entirely reserved for its own

@@ -79,6 +79,9 @@ def _load():
     L.oc_quantize_layer.argtypes = [vp, i64, i64, vp, vp, i64, f32, f32, i32, i32, i32, vp, vp, vp, vp,
                                     vp, vp, vp]
     L.oc_quantize_layer.restype = i32
+    L.oc_quantize_layer_group.argtypes = [i32, vp, vp, i64, vp, vp, i64, f32, f32, i32, i32, i32, vp, vp,
+                                          vp, vp, vp, vp, vp]
+    L.oc_quantize_layer_group.restype = i32
     return L
 
 
@@ -264,3 +267,43 @@ def oc_quantize_layer(W, X, Xhat, alpha, damp, wbits, groupsize, act_order, H=No
         _dev_ptr(zeros, torch.float32, "zeros", (m, ng)), pp, _stream_handle(stream))
     _check(st, "oc_quantize_layer")
     return H, W_out, codes, scales, zeros, perm_out
+
+
+def oc_quantize_layer_group(Ws, X, Xhat, alpha, damp, wbits, groupsize, act_order, H=None, W_outs=None,
+                            codes=None, scales=None, zeros=None, perm_out=None, stream=None):
+    """Hessian + QEP + GPTQ of several layers fed the same X, Xhat (one Hessian,
+    one cross term and one factorisation for all).  Ws: list of fp32 [m_l x n]
+    tensors.  Returns (H, W_outs, codes, scales, zeros, perm_out) with lists."""
+    import torch
+    count = len(Ws)
+    n = Ws[0].shape[1]
+    n_tok = X.shape[0]
+    G = n if groupsize == -1 else int(groupsize)
+    ng = max(1, n // G)
+    dev = Ws[0].device
+    ms = [int(W.shape[0]) for W in Ws]
+    if H is None:
+        H = torch.empty(n, n, dtype=torch.float32, device=dev)
+    if W_outs is None:
+        W_outs = [torch.empty_like(W) for W in Ws]
+    if codes is None:
+        codes = [torch.empty(m, n * wbits // 32, dtype=torch.int32, device=dev) for m in ms]
+    if scales is None:
+        scales = [torch.empty(m, ng, dtype=torch.float32, device=dev) for m in ms]
+    if zeros is None:
+        zeros = [torch.empty(m, ng, dtype=torch.float32, device=dev) for m in ms]
+    ptrs = lambda xs: (ctypes.c_void_p * count)(*xs)
+    w_p = ptrs([_dev_ptr(W, torch.float32, "W", (m, n)) for W, m in zip(Ws, ms)])
+    wo_p = ptrs([_dev_ptr(W, torch.float32, "W_out", (m, n)) for W, m in zip(W_outs, ms)])
+    c_p = ptrs([_dev_ptr(c, torch.int32, "codes", (m, n * wbits // 32)) for c, m in zip(codes, ms)])
+    s_p = ptrs([_dev_ptr(x, torch.float32, "scales", (m, ng)) for x, m in zip(scales, ms)])
+    z_p = ptrs([_dev_ptr(x, torch.float32, "zeros", (m, ng)) for x, m in zip(zeros, ms)])
+    m_arr = (ctypes.c_int64 * count)(*ms)
+    pp = _dev_ptr(perm_out, torch.int32, "perm_out", (n,)) if perm_out is not None else None
+    st = _lib().oc_quantize_layer_group(
+        count, w_p, m_arr, n, _dev_ptr(X, torch.bfloat16, "X", (n_tok, n)),
+        _dev_ptr(Xhat, torch.bfloat16, "Xhat", (n_tok, n)), n_tok, float(alpha), float(damp), int(wbits),
+        int(groupsize), 1 if act_order else 0, _dev_ptr(H, torch.float32, "H", (n, n)), wo_p, c_p, s_p, z_p, pp,
+        _stream_handle(stream))
+    _check(st, "oc_quantize_layer_group")
+    return H, W_outs, codes, scales, zeros, perm_out

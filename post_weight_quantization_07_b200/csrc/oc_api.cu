@@ -246,6 +246,219 @@ void gptq_sweep_and_pack(const Ctx& c, float* Wp, int64_t m, int64_t n, const fl
                "copy perm");
 }
 
+// Hessian + QEP + GPTQ of `count` layers that read the same inputs X, Xhat
+// (q/k/v of one attention block, gate/up of one MLP): H, d and the inverse
+// factor U depend only on the inputs and are made once; W d, the QEP apply
+// and GPTQ run per layer.  W[l], W_out[l], codes[l], scales[l], zeros[l] are
+// the l-th layer's device buffers (m[l] rows each).
+int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n, const void* X, const void* Xhat,
+                   int64_t n_tok, float alpha, float damp, int wbits, int groupsize, int act_order, float* H,
+                   float* const* W_out, uint32_t* const* codes, float* const* scales, float* const* zeros,
+                   int32_t* perm_out, void* stream) {
+  if (count < 1 || count > kMaxGroup) fail(OC_ERR_INVALID_ARG, "count must be 1..%d", kMaxGroup);
+  if (!W || !m || !W_out || !codes || !scales || !zeros) fail(OC_ERR_INVALID_ARG, "layer arrays must be non-null");
+  int64_t m_max = 0;
+  for (int l = 0; l < count; ++l) {
+    check_gptq_args(W[l], m[l], n, wbits, groupsize, damp, act_order, codes[l], scales[l], zeros[l]);
+    if (!W_out[l]) fail(OC_ERR_INVALID_ARG, "W_out[%d] must be non-null", l);
+    if (!aligned16(W_out[l])) fail(OC_ERR_INVALID_ARG, "W_out[%d] must be 16-byte aligned", l);
+    for (int k = 0; k < count; ++k)
+      if (W_out[l] == W[k]) fail(OC_ERR_INVALID_ARG, "W_out[%d] must not alias an input weight", l);
+    m_max = std::max(m_max, m[l]);
+  }
+  if (!X || !Xhat || !H) fail(OC_ERR_INVALID_ARG, "X, Xhat, H must be non-null");
+  if (n_tok < 1 || n_tok > (int64_t(1) << 31) - 64) fail(OC_ERR_INVALID_ARG, "n_tok out of range");
+  if (!(alpha == alpha) || alpha > 3.4e38f || alpha < -3.4e38f) fail(OC_ERR_INVALID_ARG, "alpha must be finite");
+  if (!aligned16(X) || !aligned16(Xhat) || !aligned16(H)) fail(OC_ERR_INVALID_ARG, "X, Xhat, H must be 16-byte aligned");
+  const int64_t G = (groupsize == -1) ? n : groupsize;
+  Ctx c = make_ctx(stream);
+  const size_t nn = static_cast<size_t>(n) * n, mn = static_cast<size_t>(m_max) * n;
+  Carve sizing{nullptr};
+  sizing.take<float>(nn);                 // d -> U
+  sizing.take<float>(nn);                 // d^T hi -> U hi
+  sizing.take<float>(nn + 4096);          // d^T lo -> U lo
+  sizing.take<float>(nn);                 // factor input -> U -> U^T hi
+  sizing.take<float>(nn);                 // inverse factor -> U^T lo
+  sizing.take<float>(nn + 4096);          // factor recursion scratch
+  sizing.take<float>(mn);                 // hi halves (W, G, T)
+  sizing.take<float>(mn);                 // lo halves
+  sizing.take<float>(mn * count);         // G -> T, one per layer
+  sizing.take<float>(mn);                 // permuted working copy of W
+  sizing.take<unsigned char>(mn);         // codes, processing order
+  sizing.take<float>(3 * static_cast<size_t>(m_max) * 128);  // block errors and their halves
+  sizing.take<int32_t>(2 * static_cast<size_t>(n));          // order | inverse
+  sizing.take<unsigned char>(n);          // dead-column mask
+  sizing.take<float>(factor_split_floats(n));
+  sizing.take<DiagStats>(1);
+  Carve cv{workspace(c, sizing.off + 256)};
+  float* D = cv.take<float>(nn);
+  float* Xi = cv.take<float>(nn);
+  float* scratch = cv.take<float>(nn + 4096);
+  float* UTh = cv.take<float>(nn);
+  float* UTl = cv.take<float>(nn);
+  float* Fs = cv.take<float>(nn + 4096);
+  float* Ph = cv.take<float>(mn);
+  float* Pl = cv.take<float>(mn);
+  float* Gs = cv.take<float>(mn * count);
+  float* Wp = cv.take<float>(mn);
+  unsigned char* codes8 = cv.take<unsigned char>(mn);
+  float* Err = cv.take<float>(3 * static_cast<size_t>(m_max) * 128);
+  float* Errh = Err + static_cast<size_t>(m_max) * 128;
+  float* Errl = Errh + static_cast<size_t>(m_max) * 128;
+  int32_t* perm = cv.take<int32_t>(2 * static_cast<size_t>(n));
+  unsigned char* dead = cv.take<unsigned char>(n);
+  float* fsplit = cv.take<float>(factor_split_floats(n));
+  DiagStats* stats = cv.take<DiagStats>(1);
+  auto Gl = [&](int l) { return Gs + static_cast<size_t>(l) * mn; };
+  const size_t nn_bytes = nn * sizeof(float);
+
+  {
+    PhaseScope ps(c, kPhHessianFix);
+    check_cuda(cudaMemsetAsync(H, 0, nn_bytes, c.stream), "memset H");
+  }
+  {
+    PhaseScope ps(c, kPhHessian);
+    launch_atb_bf16(c, Xhat, Xhat, n_tok, n, n, 2.0f, H, n, true);
+  }
+  {
+    PhaseScope ps(c, kPhHessianFix);
+    launch_mirror_upper(c, H, n);
+  }
+  // GPTQ's dampened Hessian equals QEP's 2A unless a column is dead (their
+  // dampening constants then differ): one device-to-host read decides.
+  launch_diag_stats(c, H, n, damp, 1.0f, true, stats, dead);
+  DiagStats hs{};
+  check_cuda(cudaMemcpyAsync(&hs, stats, sizeof(DiagStats), cudaMemcpyDeviceToHost, c.stream), "read stats");
+  check_cuda(cudaStreamSynchronize(c.stream), "cudaStreamSynchronize");
+  if (hs.nonfinite) return finish(c);
+  // The factorisation needs only H.  With no dead column (one factorisation
+  // serves QEP and GPTQ) it runs on a side stream, on a few SMs, while the
+  // cross product X^T Xhat occupies the rest; it factors into UTh (input
+  // reversed and dampened, output U) with UTl and Fs as its scratch.
+  const bool shared_factor = hs.n_dead == 0;
+  SideStream& ss = side_stream(c.device);
+  Ctx cs = c;
+  cs.stream = ss.stream;
+  if (shared_factor) {
+    check_cuda(cudaEventRecord(ss.fork, c.stream), "cudaEventRecord(fork)");
+    check_cuda(cudaStreamWaitEvent(cs.stream, ss.fork, 0), "cudaStreamWaitEvent(fork)");
+    PhaseScope ps(cs, kPhFactor);
+    if (act_order) launch_act_order_perm(cs, H, n, perm);
+    else launch_identity_perm(cs, n, perm);
+    launch_build_reversed(cs, H, n, perm, stats, 1.0f, true, UTh);
+    factor_inverse_upper(cs, UTh, UTl, Fs, UTh, n, true, fsplit);
+    check_cuda(cudaEventRecord(ss.join, cs.stream), "cudaEventRecord(join)");
+  }
+  {
+    PhaseScope ps(c, kPhQepCrossFix);
+    check_cuda(cudaMemsetAsync(D, 0, nn_bytes, c.stream), "memset d");
+  }
+  {
+    PhaseScope ps(c, kPhQepCross);
+    if (shared_factor) {
+      // In token ranges: between two launches the high-priority factorisation
+      // can take the freed SMs for its wide tensor-core products.
+      const int64_t parts = std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens));
+      const int64_t per = ((n_tok + parts - 1) / parts + 63) / 64 * 64;
+      const unsigned char* xb = static_cast<const unsigned char*>(X);
+      const unsigned char* hb = static_cast<const unsigned char*>(Xhat);
+      for (int64_t t0 = 0; t0 < n_tok; t0 += per) {
+        const int64_t len = std::min(per, n_tok - t0);
+        launch_atb_bf16(c, xb + t0 * n * 2, hb + t0 * n * 2, len, n, n, 1.0f, D, n, false, c.sm_count - kSideSMs);
+      }
+    } else {
+      launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false, 0);
+    }
+  }
+  {
+    PhaseScope ps(c, kPhQepCrossFix);
+    launch_sub_half(c, D, H, n);
+  }
+  {
+    // G = W d for every layer while the split copies of d^T are live
+    PhaseScope ps(c, kPhQepWDelta);
+    split_tf32(c, D, n, n, n, Xi, scratch, n, true);
+    for (int l = 0; l < count; ++l) {
+      split_tf32(c, W[l], m[l], n, n, Ph, Pl, n);
+      gemm_tf32x3(c, m[l], n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, Gl(l), n, kANone);
+    }
+  }
+  if (!shared_factor) {
+    // two factorisations: QEP's own (original order), then GPTQ's
+    {
+      PhaseScope ps(c, kPhFactor);
+      DiagStats* qs = stats;
+      launch_diag_stats(c, H, n, damp, 1.0f, false, qs, nullptr);
+      launch_build_reversed(c, H, n, nullptr, qs, 1.0f, false, D);
+      factor_inverse_upper(c, D, Xi, scratch, D, n, true, fsplit);
+    }
+    {
+      PhaseScope ps(c, kPhQepApply);
+      split_tf32(c, D, n, n, n, Xi, scratch, n);
+      split_tf32(c, D, n, n, n, UTh, UTl, n, true);
+      for (int l = 0; l < count; ++l) {
+        const size_t ml = static_cast<size_t>(m[l]) * n;
+        split_tf32(c, Gl(l), m[l], n, n, Ph, Pl, n);
+        gemm_tf32x3(c, m[l], n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, Gl(l), n, kBLower);
+        split_tf32(c, Gl(l), m[l], n, n, Ph, Pl, n);
+        launch_copy_f32(c, W[l], W_out[l], static_cast<int64_t>(ml));
+        gemm_tf32x3(c, m[l], n, n, 2.f * alpha, Ph, Pl, n, UTh, UTl, n, true, W_out[l], n, kBUpper);
+      }
+    }
+    {
+      PhaseScope ps(c, kPhFactor);
+      launch_diag_stats(c, H, n, damp, 1.0f, true, stats, dead);
+      if (act_order) launch_act_order_perm(c, H, n, perm);
+      else launch_identity_perm(c, n, perm);
+      launch_build_reversed(c, H, n, perm, stats, 1.0f, true, D);
+      factor_inverse_upper(c, D, Xi, scratch, D, n, true, fsplit);
+    }
+    {
+      PhaseScope ps(c, kPhGptqPrep);
+      split_tf32(c, D, n, n, n, UTh, UTl, n, true);
+    }
+    for (int l = 0; l < count; ++l) {
+      {
+        PhaseScope ps(c, kPhGptqPrep);
+        launch_permute_w(c, W_out[l], m[l], n, perm, dead, Wp);
+        if (act_order) launch_static_grid(c, W_out[l], m[l], n, static_cast<int>(G), wbits, dead, scales[l], zeros[l]);
+      }
+      gptq_sweep_and_pack(c, Wp, m[l], n, D, UTh, UTl, static_cast<int>(G), wbits, act_order != 0, perm, scales[l],
+                          zeros[l], codes8, Err, Errh, Errl, codes[l], l == 0 ? perm_out : nullptr);
+    }
+    return finish(c);
+  }
+
+  check_cuda(cudaStreamWaitEvent(c.stream, ss.join, 0), "cudaStreamWaitEvent(join)");
+  {
+    PhaseScope ps(c, kPhQepApply);
+    check_cuda(cudaMemcpyAsync(D, UTh, nn_bytes, cudaMemcpyDeviceToDevice, c.stream), "copy U");
+    split_tf32(c, D, n, n, n, Xi, scratch, n);
+    split_tf32(c, D, n, n, n, UTh, UTl, n, true);
+    launch_invert_perm(c, perm, n);
+  }
+  for (int l = 0; l < count; ++l) {
+    // QEP applied in processing order: W'P = WP + 2 alpha ((G P) U^T) U
+    {
+      PhaseScope ps(c, kPhQepApply);
+      launch_permute_w(c, Gl(l), m[l], n, perm, dead, Wp);             // G P
+      split_tf32(c, Wp, m[l], n, n, Ph, Pl, n);
+      gemm_tf32x3(c, m[l], n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, Gl(l), n, kBLower);  // T = (G P) U^T
+      split_tf32(c, Gl(l), m[l], n, n, Ph, Pl, n);
+      launch_permute_w(c, W[l], m[l], n, perm, dead, Wp);              // W P
+      gemm_tf32x3(c, m[l], n, n, 2.f * alpha, Ph, Pl, n, UTh, UTl, n, true, Wp, n, kBUpper);
+      launch_permute_w(c, Wp, m[l], n, perm + n, dead, W_out[l]);      // back to original order
+    }
+    if (act_order) {
+      PhaseScope ps(c, kPhGptqPrep);
+      launch_static_grid(c, W_out[l], m[l], n, static_cast<int>(G), wbits, dead, scales[l], zeros[l]);
+    }
+    gptq_sweep_and_pack(c, Wp, m[l], n, D, UTh, UTl, static_cast<int>(G), wbits, act_order != 0, perm, scales[l],
+                        zeros[l], codes8, Err, Errh, Errl, codes[l], l == 0 ? perm_out : nullptr);
+  }
+  return finish(c);
+}
+
 }  // namespace
 }  // namespace oc
 
@@ -497,181 +710,18 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
                       float alpha, float damp, int wbits, int groupsize, int act_order, float* H, float* W_out,
                       uint32_t* codes, float* scales, float* zeros, int32_t* perm_out, void* stream) {
   return guarded([&]() -> int {
-    check_gptq_args(W, m, n, wbits, groupsize, damp, act_order, codes, scales, zeros);
-    if (!X || !Xhat || !H || !W_out) fail(OC_ERR_INVALID_ARG, "X, Xhat, H, W_out must be non-null");
-    if (W_out == W) fail(OC_ERR_INVALID_ARG, "W_out must not alias W");
-    if (n_tok < 1 || n_tok > (int64_t(1) << 31) - 64) fail(OC_ERR_INVALID_ARG, "n_tok out of range");
-    if (!(alpha == alpha) || alpha > 3.4e38f || alpha < -3.4e38f) fail(OC_ERR_INVALID_ARG, "alpha must be finite");
-    if (!aligned16(X) || !aligned16(Xhat) || !aligned16(H) || !aligned16(W_out))
-      fail(OC_ERR_INVALID_ARG, "X, Xhat, H, W_out must be 16-byte aligned");
-    const int64_t G = (groupsize == -1) ? n : groupsize;
-    Ctx c = make_ctx(stream);
-    const size_t nn = static_cast<size_t>(n) * n, mn = static_cast<size_t>(m) * n;
-    Carve sizing{nullptr};
-    sizing.take<float>(nn);                 // d -> M -> U
-    sizing.take<float>(nn);                 // d^T hi -> inverse factor -> U hi
-    sizing.take<float>(nn + 4096);          // d^T lo -> recursion scratch -> U lo
-    sizing.take<float>(nn);                 // factor input -> U -> U^T hi
-    sizing.take<float>(nn);                 // inverse factor -> U^T lo
-    sizing.take<float>(nn + 4096);          // factor recursion scratch
-    sizing.take<float>(mn);                 // hi halves (W, G, T)
-    sizing.take<float>(mn);                 // lo halves
-    sizing.take<float>(mn);                 // G -> T
-    sizing.take<float>(mn);                 // permuted working copy of W
-    sizing.take<unsigned char>(mn);         // codes, processing order
-    sizing.take<float>(3 * static_cast<size_t>(m) * 128);  // block errors and their halves
-    sizing.take<int32_t>(2 * static_cast<size_t>(n));      // order | inverse
-    sizing.take<unsigned char>(n);          // dead-column mask
-    sizing.take<float>(factor_split_floats(n));
-    sizing.take<DiagStats>(1);
-    Carve cv{workspace(c, sizing.off + 256)};
-    float* D = cv.take<float>(nn);
-    float* Xi = cv.take<float>(nn);
-    float* scratch = cv.take<float>(nn + 4096);
-    float* UTh = cv.take<float>(nn);
-    float* UTl = cv.take<float>(nn);
-    float* Fs = cv.take<float>(nn + 4096);
-    float* Ph = cv.take<float>(mn);
-    float* Pl = cv.take<float>(mn);
-    float* G2 = cv.take<float>(mn);
-    float* Wp = cv.take<float>(mn);
-    unsigned char* codes8 = cv.take<unsigned char>(mn);
-    float* Err = cv.take<float>(3 * static_cast<size_t>(m) * 128);
-    float* Errh = Err + static_cast<size_t>(m) * 128;
-    float* Errl = Errh + static_cast<size_t>(m) * 128;
-    int32_t* perm = cv.take<int32_t>(2 * static_cast<size_t>(n));
-    unsigned char* dead = cv.take<unsigned char>(n);
-    float* fsplit = cv.take<float>(factor_split_floats(n));
-    DiagStats* stats = cv.take<DiagStats>(1);
+    return quantize_group(1, &W, &m, n, X, Xhat, n_tok, alpha, damp, wbits, groupsize, act_order, H, &W_out, &codes,
+                          &scales, &zeros, perm_out, stream);
+  });
+}
 
-    {
-      PhaseScope ps(c, kPhHessianFix);
-      check_cuda(cudaMemsetAsync(H, 0, nn * sizeof(float), c.stream), "memset H");
-    }
-    {
-      PhaseScope ps(c, kPhHessian);
-      launch_atb_bf16(c, Xhat, Xhat, n_tok, n, n, 2.0f, H, n, true);
-    }
-    {
-      PhaseScope ps(c, kPhHessianFix);
-      launch_mirror_upper(c, H, n);
-    }
-    // GPTQ's dampened Hessian equals QEP's 2A unless a column is dead (their
-    // dampening constants then differ): one device-to-host read decides.
-    launch_diag_stats(c, H, n, damp, 1.0f, true, stats, dead);
-    DiagStats hs{};
-    check_cuda(cudaMemcpyAsync(&hs, stats, sizeof(DiagStats), cudaMemcpyDeviceToHost, c.stream), "read stats");
-    check_cuda(cudaStreamSynchronize(c.stream), "cudaStreamSynchronize");
-    if (hs.nonfinite) return finish(c);
-    // The factorisation needs only H.  With no dead column (one factorisation
-    // serves QEP and GPTQ) it runs on a side stream, on a few SMs, while the
-    // cross product X^T Xhat occupies the rest; it factors into UTh (input
-    // reversed and dampened, output U) with UTl and Fs as its scratch.
-    const bool shared_factor = hs.n_dead == 0;
-    SideStream& ss = side_stream(c.device);
-    Ctx cs = c;
-    cs.stream = ss.stream;
-    if (shared_factor) {
-      check_cuda(cudaEventRecord(ss.fork, c.stream), "cudaEventRecord(fork)");
-      check_cuda(cudaStreamWaitEvent(cs.stream, ss.fork, 0), "cudaStreamWaitEvent(fork)");
-      PhaseScope ps(cs, kPhFactor);
-      if (act_order) launch_act_order_perm(cs, H, n, perm);
-      else launch_identity_perm(cs, n, perm);
-      launch_build_reversed(cs, H, n, perm, stats, 1.0f, true, UTh);
-      factor_inverse_upper(cs, UTh, UTl, Fs, UTh, n, true, fsplit);
-      check_cuda(cudaEventRecord(ss.join, cs.stream), "cudaEventRecord(join)");
-    }
-    {
-      PhaseScope ps(c, kPhQepCrossFix);
-      check_cuda(cudaMemsetAsync(D, 0, nn * sizeof(float), c.stream), "memset d");
-    }
-    {
-      PhaseScope ps(c, kPhQepCross);
-      if (shared_factor) {
-        // In token ranges: between two launches the high-priority factorisation
-        // can take the freed SMs for its wide tensor-core products.
-        const int64_t parts = std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens));
-        const int64_t per = ((n_tok + parts - 1) / parts + 63) / 64 * 64;
-        const unsigned char* xb = static_cast<const unsigned char*>(X);
-        const unsigned char* hb = static_cast<const unsigned char*>(Xhat);
-        for (int64_t t0 = 0; t0 < n_tok; t0 += per) {
-          const int64_t len = std::min(per, n_tok - t0);
-          launch_atb_bf16(c, xb + t0 * n * 2, hb + t0 * n * 2, len, n, n, 1.0f, D, n, false,
-                          c.sm_count - kSideSMs);
-        }
-      } else {
-        launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false, 0);
-      }
-    }
-    {
-      PhaseScope ps(c, kPhQepCrossFix);
-      launch_sub_half(c, D, H, n);
-    }
-    {
-      PhaseScope ps(c, kPhQepWDelta);
-      split_tf32(c, D, n, n, n, Xi, scratch, n, true);
-      split_tf32(c, W, m, n, n, Ph, Pl, n);
-      gemm_tf32x3(c, m, n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, G2, n, kANone);
-    }
-    if (!shared_factor) {
-      // two factorisations: QEP's own (original order), then GPTQ's
-      {
-        PhaseScope ps(c, kPhFactor);
-        DiagStats* qs = stats;
-        launch_diag_stats(c, H, n, damp, 1.0f, false, qs, nullptr);
-        launch_build_reversed(c, H, n, nullptr, qs, 1.0f, false, D);
-        factor_inverse_upper(c, D, Xi, scratch, D, n, true, fsplit);
-      }
-      {
-        PhaseScope ps(c, kPhQepApply);
-        split_tf32(c, D, n, n, n, Xi, scratch, n);
-        split_tf32(c, D, n, n, n, UTh, UTl, n, true);
-        split_tf32(c, G2, m, n, n, Ph, Pl, n);
-        gemm_tf32x3(c, m, n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, G2, n, kBLower);
-        split_tf32(c, G2, m, n, n, Ph, Pl, n);
-        launch_copy_f32(c, W, W_out, static_cast<int64_t>(mn));
-        gemm_tf32x3(c, m, n, n, 2.f * alpha, Ph, Pl, n, UTh, UTl, n, true, W_out, n, kBUpper);
-      }
-      {
-        PhaseScope ps(c, kPhFactor);
-        launch_diag_stats(c, H, n, damp, 1.0f, true, stats, dead);
-        if (act_order) launch_act_order_perm(c, H, n, perm);
-        else launch_identity_perm(c, n, perm);
-        launch_build_reversed(c, H, n, perm, stats, 1.0f, true, D);
-        factor_inverse_upper(c, D, Xi, scratch, D, n, true, fsplit);
-      }
-      {
-        PhaseScope ps(c, kPhGptqPrep);
-        split_tf32(c, D, n, n, n, UTh, UTl, n, true);
-        launch_permute_w(c, W_out, m, n, perm, dead, Wp);
-        if (act_order) launch_static_grid(c, W_out, m, n, static_cast<int>(G), wbits, dead, scales, zeros);
-      }
-    } else {
-      check_cuda(cudaStreamWaitEvent(c.stream, ss.join, 0), "cudaStreamWaitEvent(join)");
-      // QEP applied in processing order: W'P = WP + 2 alpha ((G P) U^T) U
-      {
-        PhaseScope ps(c, kPhQepApply);
-        check_cuda(cudaMemcpyAsync(D, UTh, nn * sizeof(float), cudaMemcpyDeviceToDevice, c.stream), "copy U");
-        const float* U = D;
-        split_tf32(c, U, n, n, n, Xi, scratch, n);
-        split_tf32(c, U, n, n, n, UTh, UTl, n, true);
-        launch_permute_w(c, G2, m, n, perm, dead, Wp);           // G P
-        split_tf32(c, Wp, m, n, n, Ph, Pl, n);
-        gemm_tf32x3(c, m, n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, G2, n, kBLower);  // T = (G P) U^T
-        split_tf32(c, G2, m, n, n, Ph, Pl, n);
-        launch_permute_w(c, W, m, n, perm, dead, Wp);            // W P
-        gemm_tf32x3(c, m, n, n, 2.f * alpha, Ph, Pl, n, UTh, UTl, n, true, Wp, n, kBUpper);
-        launch_invert_perm(c, perm, n);
-        launch_permute_w(c, Wp, m, n, perm + n, dead, W_out);    // back to original order
-      }
-      if (act_order) {
-        PhaseScope ps(c, kPhGptqPrep);
-        launch_static_grid(c, W_out, m, n, static_cast<int>(G), wbits, dead, scales, zeros);
-      }
-    }
-    gptq_sweep_and_pack(c, Wp, m, n, D, UTh, UTl, static_cast<int>(G), wbits, act_order != 0, perm, scales, zeros,
-                        codes8, Err, Errh, Errl, codes, perm_out);
-    return finish(c);
+int oc_quantize_layer_group(int count, const float* const* W, const int64_t* m, int64_t n, const void* X,
+                            const void* Xhat, int64_t n_tok, float alpha, float damp, int wbits, int groupsize,
+                            int act_order, float* H, float* const* W_out, uint32_t* const* codes,
+                            float* const* scales, float* const* zeros, int32_t* perm_out, void* stream) {
+  return guarded([&]() -> int {
+    return quantize_group(count, W, m, n, X, Xhat, n_tok, alpha, damp, wbits, groupsize, act_order, H, W_out, codes,
+                          scales, zeros, perm_out, stream);
   });
 }
 

@@ -108,6 +108,8 @@ struct SideStream {
 SideStream& side_stream(int device);
 // SMs left to the side stream while the main stream's product runs.
 constexpr int kSideSMs = 8;
+// Most layers one oc_quantize_layer_group call takes.
+constexpr int kMaxGroup = 16;
 // The cross product beside it runs as up to kCrossParts launches over token
 // ranges of at least kCrossPartMinTokens tokens each.
 constexpr int64_t kCrossParts = 32;

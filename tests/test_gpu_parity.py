@@ -320,3 +320,64 @@ def test_fused_layer_matches_oracle(m, n, n_tok, wbits, G, act, dead):
     assert st["scale_max_rel"] <= SCALE_TOL, st
     ident = level_identity(cg, zg, ref["codes"], ref["zeros"], G)
     assert ident >= code_frac_for(cg.size), (ident, st)
+
+
+# ----------------------------------------------------------------------------- layer groups
+
+@pytest.mark.parametrize("ms,n,n_tok,wbits,G,act,dead", [
+    ((256, 128, 384), 512, 2048, 4, 128, False, False),
+    ((96, 200), 384, 1500, 3, 64, True, False),
+    ((64, 128, 32), 256, 1024, 4, 64, True, True),   # dead columns: two factorisations
+])
+def test_layer_group_matches_oracle_per_layer(ms, n, n_tok, wbits, G, act, dead):
+    # Layers fed the same inputs share H, d and the factor; each must match
+    # the oracle run on that layer alone.
+    L = random_layer_host(max(ms), n, n_tok, seed=5000 + n)
+    X, Xh = L["X"].copy(), L["Xhat"].copy()
+    if dead:
+        X[:, [3, 50]] = 0.0
+        Xh[:, [3, 50]] = 0.0
+    rng = np.random.default_rng(77)
+    Ws = [(0.02 * rng.standard_normal((m, n))).astype(np.float32) for m in ms]
+    Ho = oracle.hessian(Xh)
+    perm = torch.empty(n, dtype=torch.int32, device="cuda")
+    Hg, Wouts, codes, scales, zeros, _ = oc.oc_quantize_layer_group(
+        [dev(W) for W in Ws], bf16_dev(X), bf16_dev(Xh), 0.5, 0.01, wbits, G, act, perm_out=perm)
+    torch.cuda.synchronize()
+    assert rel_fro(Hg.cpu().numpy(), Ho) <= H_TOL
+    pg = perm.cpu().numpy()
+    for l, W in enumerate(Ws):
+        W64 = W.astype(np.float64)
+        Wpo = oracle.qep_correct(W64, X, Xh, 0.5, 0.01, H=Ho)
+        ref = oracle.gptq_quantize(Wpo, Ho, wbits, G, 0.01, act)
+        assert np.abs(Wouts[l].cpu().numpy() - Wpo).max() <= QEP_TOL * np.abs(W64).max(), l
+        cg = oracle.unpack_codes(codes[l].cpu().numpy().view(np.uint32), wbits, n)
+        sg, zg = scales[l].cpu().numpy(), zeros[l].cpu().numpy()
+        st = oracle.teacher_forced_check(Wpo, Ho, wbits, G, 0.01, act, cg, sg, zg, perm=pg)
+        assert st["n_bad"] == 0 and st["zero_bad"] == 0, (l, st)
+        assert st["scale_max_rel"] <= SCALE_TOL, (l, st)
+        ident = level_identity(cg, zg, ref["codes"], ref["zeros"], G)
+        assert ident >= code_frac_for(cg.size), (l, ident, st)
+
+
+def test_layer_group_of_one_is_the_layer_call():
+    L = random_layer_host(192, 256, 1024, seed=5101)
+    W, X, Xh = dev(L["W"]), bf16_dev(L["X"]), bf16_dev(L["Xhat"])
+    _, Wa, ca, sa, za, _ = oc.oc_quantize_layer(W, X, Xh, 0.5, 0.01, 4, 64, True)
+    _, Wb, cb, sb, zb, _ = oc.oc_quantize_layer_group([W], X, Xh, 0.5, 0.01, 4, 64, True)
+    torch.cuda.synchronize()
+    # same kernels in the same order; only the order of fp32 additions inside
+    # the tensor-core reduction may differ between runs
+    assert torch.allclose(Wa, Wb[0], rtol=0, atol=1e-6 * float(Wa.abs().max()))
+    same = float((ca == cb[0]).float().mean())
+    assert same >= 0.99
+    assert torch.allclose(sa, sb[0], rtol=1e-5, atol=0)
+
+
+def test_layer_group_rejects_bad_arguments():
+    L = random_layer_host(64, 128, 512, seed=5102)
+    W, X, Xh = dev(L["W"]), bf16_dev(L["X"]), bf16_dev(L["Xhat"])
+    with pytest.raises(oc.OcError):
+        oc.oc_quantize_layer_group([W, W], X, Xh, 0.5, 0.01, 4, 64, False, W_outs=[W.clone(), W])
+    with pytest.raises(oc.OcError):
+        oc.oc_quantize_layer_group([W] * 17, X, Xh, 0.5, 0.01, 4, 64, False)
