@@ -204,6 +204,21 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
                       float* zeros, int32_t* perm_out, void* stream);
 
 /*
+ * Dequantise packed GPTQ output: out[i][j] = scales[i][g] * (q[i][j] - zeros[i][g]),
+ * g = j / groupsize, q read from row i's LSB-first bitstream of wbits-bit codes
+ * (the layout oc_gptq_quantize writes).  This is the weight the quantised
+ * layer applies (One Compression hub page, section "核心功能拆解": the
+ * quantised model's layers); it feeds the next layer's calibration inputs when
+ * quantisation error is propagated through a chain of layers.
+ *   codes   uint32 [m x n*wbits/32];  scales, zeros fp32 [m x n/groupsize].
+ *   out     [m x n], fp32 (out_bf16 = 0) or bf16 rounded to nearest even (1).
+ * Errors: OC_ERR_INVALID_ARG for null pointers, wbits outside 2..4, n*wbits
+ * not a multiple of 32, or a groupsize that does not divide n.
+ */
+int oc_dequantize(const uint32_t* codes, const float* scales, const float* zeros, int64_t m, int64_t n,
+                  int wbits, int groupsize, void* out, int out_bf16, void* stream);
+
+/*
  * Several layers that read the same calibration inputs, e.g. the q, k and v
  * projections of one attention block or gate and up of one MLP (the One
  * Compression hub page, section "核心功能拆解", quantises a model layer by

@@ -489,3 +489,60 @@ def teacher_forced_check(W, H, wbits: int, groupsize: int, damp: float, act_orde
         if b1 < n:
             W1[:, b1:] -= Eb @ U[b0:b1, b1:]
     return stats
+
+
+# ----------------------------------------------------------------------------- propagation chain
+
+def dequantize(packed, scales, zeros, wbits: int, groupsize: int, n: int):
+    """Q = scale * (q - zero) from packed codes (original column order)."""
+    codes = unpack_codes(np.asarray(packed), wbits, n)
+    G = _group_size(groupsize, n)
+    s = np.repeat(_f64(scales), G, axis=1)
+    z = np.repeat(_f64(zeros), G, axis=1)
+    return s * (codes - z)
+
+
+def _bf16(a):
+    """Round to the nearest bf16 value (ties to even), as float64."""
+    a32 = np.ascontiguousarray(a, dtype=np.float32)
+    u = a32.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
+    return r.view(np.float32).astype(np.float64)
+
+
+def _act(y, act: str):
+    if act == "silu":
+        return y / (1.0 + np.exp(-y))
+    if act == "none":
+        return y
+    raise ValueError(act)
+
+
+def quantize_chain(Ws, x0, alpha: float, damp: float, wbits: int, groupsize: int, act_order: bool,
+                   act: str = "silu"):
+    """Quantise a chain of linear layers with true error propagation (QEP's
+    setting, OneComp release summary section "量化錯誤傳播 (QEP)").
+
+    Layer l maps d_in = Ws[l].shape[1] features to d_out = Ws[l].shape[0].  Two
+    activation streams run through the chain: the full-precision one,
+    X_{l+1} = f(X_l W_l^T), and the quantised one, Xh_{l+1} = f(Xh_l Q_l^T),
+    starting from Xh_0 = X_0.  Layer l is quantised on its own pair
+    (X_l, Xh_l): H = 2 Xh_l^T Xh_l, W' = qep_correct(W_l, X_l, Xh_l), GPTQ of W'.
+    Weights and activations enter each forward product as bf16 values, the
+    product is rounded to bf16 and so is the activation of it (a bf16 model's
+    linear layer and activation); sums are exact in float64 here.
+    Returns a list of per-layer dicts (X, Xhat, H, W_prime, codes, packed,
+    scales, zeros, deq) and the final pair (X_L, Xh_L).
+    """
+    x = _bf16(x0)
+    xh = x.copy()
+    layers = []
+    for W in Ws:
+        W = _f64(W)
+        H = hessian(xh)
+        Wp = qep_correct(W, x, xh, alpha, damp, H=H)
+        q = gptq_quantize(Wp, H, wbits, groupsize, damp, act_order)
+        layers.append({"X": x, "Xhat": xh, "H": H, "W_prime": Wp, **q})
+        x = _bf16(_act(_bf16(x @ _bf16(W).T), act))
+        xh = _bf16(_act(_bf16(xh @ _bf16(q["deq"]).T), act))
+    return layers, (x, xh)

@@ -82,6 +82,8 @@ def _load():
     L.oc_quantize_layer_group.argtypes = [i32, vp, vp, i64, vp, vp, i64, f32, f32, i32, i32, i32, vp, vp,
                                           vp, vp, vp, vp, vp]
     L.oc_quantize_layer_group.restype = i32
+    L.oc_dequantize.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, i32, vp]
+    L.oc_dequantize.restype = i32
     return L
 
 
@@ -307,3 +309,56 @@ def oc_quantize_layer_group(Ws, X, Xhat, alpha, damp, wbits, groupsize, act_orde
         _stream_handle(stream))
     _check(st, "oc_quantize_layer_group")
     return H, W_outs, codes, scales, zeros, perm_out
+
+
+def oc_dequantize(codes, scales, zeros, n, wbits, groupsize, out=None, bf16=False, stream=None):
+    """scale * (code - zero) of packed codes, [m x n] fp32 or bf16."""
+    import torch
+    m = codes.shape[0]
+    G = n if groupsize == -1 else int(groupsize)
+    dt = torch.bfloat16 if bf16 else torch.float32
+    if out is None:
+        out = torch.empty(m, n, dtype=dt, device=codes.device)
+    st = _lib().oc_dequantize(_dev_ptr(codes, torch.int32, "codes", (m, n * wbits // 32)),
+                              _dev_ptr(scales, torch.float32, "scales", (m, n // G)),
+                              _dev_ptr(zeros, torch.float32, "zeros", (m, n // G)), m, n, int(wbits),
+                              int(groupsize), _dev_ptr(out, dt, "out", (m, n)), 1 if bf16 else 0,
+                              _stream_handle(stream))
+    _check(st, "oc_dequantize")
+    return out
+
+
+def quantize_chain(Ws, X0, alpha, damp, wbits, groupsize, act_order, act="silu", stream=None):
+    """Quantise a chain of linear layers with the quantisation error propagated.
+
+    Two bf16 activation streams run through the chain, the full-precision
+    X_{l+1} = f(X_l W_l^T) and the quantised Xh_{l+1} = f(Xh_l Q_l^T) from
+    Xh_0 = X_0; layer l is quantised by oc_quantize_layer on its own pair
+    (X_l, Xh_l), so its QEP correction sees the error of every layer before it.
+    The forward products are plain bf16 GEMMs (cuBLAS through torch, fp32
+    accumulation, bf16 result), f is SiLU (act="silu") or the identity, and
+    Q_l comes from oc_dequantize.  Ws: fp32 [d_out x d_in] tensors whose
+    d_in matches the previous d_out.  Returns (layers, (X_L, Xh_L)), each
+    layer a dict with its inputs and oc_quantize_layer's outputs.
+    """
+    import torch
+    import torch.nn.functional as F
+    if act not in ("silu", "none"):
+        raise ValueError("act must be 'silu' or 'none'")
+    x = X0.to(torch.bfloat16).contiguous()
+    xh = x.clone()
+    layers = []
+    for W in Ws:
+        m, n = W.shape
+        perm = torch.empty(n, dtype=torch.int32, device=W.device)
+        H, Wp, codes, scales, zeros, _ = oc_quantize_layer(W, x, xh, alpha, damp, wbits, groupsize, act_order,
+                                                           perm_out=perm, stream=stream)
+        Q = oc_dequantize(codes, scales, zeros, n, wbits, groupsize, bf16=True, stream=stream)
+        layers.append({"X": x, "Xhat": xh, "H": H, "W_prime": Wp, "codes": codes, "scales": scales,
+                       "zeros": zeros, "perm": perm})
+        y = x @ W.to(torch.bfloat16).t()
+        yh = xh @ Q.t()
+        if act == "silu":
+            y, yh = F.silu(y), F.silu(yh)
+        x, xh = y.contiguous(), yh.contiguous()
+    return layers, (x, xh)

@@ -706,6 +706,22 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
   });
 }
 
+int oc_dequantize(const uint32_t* codes, const float* scales, const float* zeros, int64_t m, int64_t n, int wbits,
+                  int groupsize, void* out, int out_bf16, void* stream) {
+  return guarded([&]() -> int {
+    if (!codes || !scales || !zeros || !out) fail(OC_ERR_INVALID_ARG, "codes, scales, zeros, out must be non-null");
+    if (m < 1 || n < 1) fail(OC_ERR_INVALID_ARG, "m and n must be >= 1");
+    if (wbits < 2 || wbits > 4) fail(OC_ERR_INVALID_ARG, "wbits must be 2, 3 or 4");
+    if ((n * wbits) % 32) fail(OC_ERR_INVALID_ARG, "n * wbits must be a multiple of 32");
+    const int64_t G = (groupsize == -1) ? n : groupsize;
+    if (G < 1 || n % G) fail(OC_ERR_INVALID_ARG, "groupsize must divide n (or be -1)");
+    if (out_bf16 != 0 && out_bf16 != 1) fail(OC_ERR_INVALID_ARG, "out_bf16 must be 0 or 1");
+    Ctx c = make_ctx(stream);
+    launch_dequant(c, codes, scales, zeros, m, n, wbits, G, out, out_bf16 != 0);
+    return finish(c);
+  });
+}
+
 int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const void* Xhat, int64_t n_tok,
                       float alpha, float damp, int wbits, int groupsize, int act_order, float* H, float* W_out,
                       uint32_t* codes, float* scales, float* zeros, int32_t* perm_out, void* stream) {

@@ -186,6 +186,9 @@ void launch_sweep_block(const Ctx& c, float* Wp, int64_t m, int64_t n, const flo
 // Packs codes8 (processing order) into the original-order bitstream; perm2
 // holds the processing order in its first n entries and receives the inverse
 // permutation in the next n.
+// out[i][j] = scale * (code - zero), fp32 or bf16, original column order.
+void launch_dequant(const Ctx& c, const uint32_t* codes, const float* scales, const float* zeros, int64_t m,
+                    int64_t n, int wbits, int64_t G, void* out, bool bf16);
 void launch_pack(const Ctx& c, const unsigned char* codes8, int64_t m, int64_t n, int wbits,
                  int32_t* perm2, uint32_t* codes);
 

@@ -381,3 +381,67 @@ def test_layer_group_rejects_bad_arguments():
         oc.oc_quantize_layer_group([W, W], X, Xh, 0.5, 0.01, 4, 64, False, W_outs=[W.clone(), W])
     with pytest.raises(oc.OcError):
         oc.oc_quantize_layer_group([W] * 17, X, Xh, 0.5, 0.01, 4, 64, False)
+
+
+# ----------------------------------------------------------------------------- dequantisation, chains
+
+@pytest.mark.parametrize("wbits,G", [(2, 64), (3, 128), (4, 32)])
+def test_dequantize_matches_oracle(wbits, G):
+    rng = np.random.default_rng(90 + wbits)
+    m, n = 37, 512
+    codes = rng.integers(0, 1 << wbits, size=(m, n))
+    packed = oracle.pack_codes(codes, wbits).view(np.int32)
+    scales = rng.uniform(1e-3, 0.1, size=(m, n // G)).astype(np.float32)
+    zeros = rng.integers(0, 1 << wbits, size=(m, n // G)).astype(np.float32)
+    want = oracle.dequantize(packed.view(np.uint32), scales, zeros, wbits, G, n)
+    c_d = torch.from_numpy(np.ascontiguousarray(packed)).cuda()
+    s_d, z_d = dev(scales), dev(zeros)
+    out32 = oc.oc_dequantize(c_d, s_d, z_d, n, wbits, G)
+    out16 = oc.oc_dequantize(c_d, s_d, z_d, n, wbits, G, bf16=True)
+    torch.cuda.synchronize()
+    # fp32: the correctly rounded product; bf16: that rounded to nearest even
+    assert np.array_equal(out32.cpu().numpy(), want.astype(np.float32))
+    assert np.array_equal(out16.float().cpu().numpy(), oracle._bf16(want.astype(np.float32)).astype(np.float32))
+
+
+def test_chain_matches_oracle():
+    rng = np.random.default_rng(91)
+    N = 2048
+    x0 = rng.standard_normal((N, 256))
+    x0[:, :3] *= 8.0
+    x0 = oracle._bf16(x0)
+    Ws = [(rng.standard_normal((256, 256)) / 16).astype(np.float32),
+          (rng.standard_normal((192, 256)) / 16).astype(np.float32),
+          (rng.standard_normal((128, 192)) / 14).astype(np.float32)]
+    ref_layers, (xo, xho) = oracle.quantize_chain(Ws, x0, 0.5, 0.01, 4, 64, False)
+    layers, (xg, xhg) = oc.quantize_chain([dev(W) for W in Ws], dev(x0), 0.5, 0.01, 4, 64, False)
+    torch.cuda.synchronize()
+    # layer 0 sees identical inputs: the full per-layer checks
+    r0, g0 = ref_layers[0], layers[0]
+    assert rel_fro(g0["H"].cpu().numpy(), r0["H"]) <= H_TOL
+    cg = oracle.unpack_codes(g0["codes"].cpu().numpy().view(np.uint32), 4, 256)
+    st = oracle.teacher_forced_check(r0["W_prime"], r0["H"], 4, 64, 0.01, False, cg,
+                                     g0["scales"].cpu().numpy(), g0["zeros"].cpu().numpy())
+    assert st["n_bad"] == 0 and st["zero_bad"] == 0 and st["scale_max_rel"] <= SCALE_TOL, st
+    # the full-precision stream: bf16 products of identical bf16 operands
+    x1g = layers[1]["X"].float().cpu().numpy()
+    x1o = ref_layers[1]["X"]
+    assert np.mean(x1g == x1o) >= 0.99
+    assert np.abs(x1g - x1o).max() <= 2.0 ** -6 * np.abs(x1o).max()
+    # end to end: the propagated quantisation error of the chain within 1% of
+    # the oracle's
+    eg = np.linalg.norm(xg.float().cpu().numpy() - xhg.float().cpu().numpy())
+    eo = np.linalg.norm(xo - xho)
+    assert abs(eg - eo) <= 0.01 * eo, (eg, eo)
+
+
+def test_chain_qep_reduces_propagated_error_on_gpu():
+    rng = np.random.default_rng(92)
+    x0 = rng.standard_normal((4096, 128))
+    x0[:, :2] *= 8.0
+    Ws = [dev((rng.standard_normal((128, 128)) / 11).astype(np.float32)) for _ in range(4)]
+    errs = {}
+    for alpha in (0.0, 0.5):
+        _, (x, xh) = oc.quantize_chain(Ws, dev(x0), alpha, 0.01, 3, 32, False)
+        errs[alpha] = float((x.float() - xh.float()).norm() / x.float().norm())
+    assert errs[0.5] < errs[0.0], errs

@@ -395,3 +395,46 @@ def test_gptq_given_factor_equals_recomputed():
     assert np.allclose(a["scales"], b["scales"], rtol=1e-12, atol=0)
     st = oracle.teacher_forced_check(W, H, 3, 16, 0.01, True, a["codes"], a["scales"], a["zeros"], U=U)
     assert st["n_mismatch"] == 0 and st["scale_max_rel"] <= 1e-12
+
+
+def test_dequantize_inverts_pack():
+    rng = np.random.default_rng(73)
+    for wbits in (2, 3, 4):
+        codes = rng.integers(0, 1 << wbits, size=(5, 64))
+        packed = oracle.pack_codes(codes, wbits)
+        scales = rng.uniform(0.1, 1.0, size=(5, 2))
+        zeros = rng.integers(0, 1 << wbits, size=(5, 2)).astype(np.float64)
+        deq = oracle.dequantize(packed, scales, zeros, wbits, 32, 64)
+        want = np.repeat(scales, 32, axis=1) * (codes - np.repeat(zeros, 32, axis=1))
+        assert np.array_equal(deq, want)
+
+
+def test_chain_first_layer_is_plain_gptq_and_later_inputs_propagate():
+    # Xh_0 = X_0: the first layer's QEP correction vanishes (W' = W to 1e-10);
+    # the second layer's inputs are the two streams' forward products.
+    rng = np.random.default_rng(74)
+    x0 = rng.standard_normal((512, 32))
+    Ws = [0.2 * rng.standard_normal((32, 32)), 0.2 * rng.standard_normal((16, 32))]
+    layers, (x2, xh2) = oracle.quantize_chain(Ws, x0, 0.5, 0.01, 4, 16, False)
+    assert np.abs(layers[0]["W_prime"] - Ws[0]).max() <= 1e-10
+    ref = oracle.gptq_quantize(Ws[0], oracle.hessian(oracle._bf16(x0)), 4, 16, 0.01, False)
+    assert np.array_equal(layers[0]["codes"], ref["codes"])
+    x1 = layers[1]["X"]
+    want = oracle._bf16(oracle._act(oracle._bf16(oracle._bf16(x0) @ oracle._bf16(Ws[0]).T), "silu"))
+    assert np.array_equal(x1, want)
+    assert x2.shape == (512, 16) and xh2.shape == (512, 16)
+    assert not np.array_equal(layers[1]["X"], layers[1]["Xhat"])
+
+
+def test_chain_qep_reduces_propagated_error():
+    # QEP's purpose: with quantisation error arriving from earlier layers,
+    # correcting for it lowers the chain's final output error ||X_L - Xh_L||.
+    rng = np.random.default_rng(75)
+    x0 = rng.standard_normal((2048, 64))
+    x0[:, :2] *= 8.0
+    Ws = [rng.standard_normal((64, 64)) / 8.0 for _ in range(4)]
+    errs = {}
+    for alpha in (0.0, 0.5, 1.0):
+        _, (x, xh) = oracle.quantize_chain(Ws, x0, alpha, 0.01, 3, 16, False)
+        errs[alpha] = np.linalg.norm(x - xh) / np.linalg.norm(x)
+    assert errs[0.5] < errs[0.0] and errs[1.0] < errs[0.0], errs
