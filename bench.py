@@ -497,7 +497,8 @@ def run_ours(args, rank, world, local_rank):
     roof = {"bound": "tensor", "unit": "TFLOP/s", "kernel": "atb_bf16_kernel",
             "phases": gemm_phases, "peak_source": f"{peak_src} bf16 sustained (of {peak_src})",
             "achieved": round(achieved, 2), "peak": round(peak, 2),
-            "frac": round(achieved / peak, 4), "traffic": TRAFFIC_PER_LAUNCH.get(spec.name),
+            "frac": round(achieved / peak, 4),
+            "traffic": None if args.n_tok else TRAFFIC_PER_LAUNCH.get(spec.name),
             "per_launch": {"amount": per_launch, "unit": "flop", "ms": round(ms_launch, 4)}}
     sm_mhz = clocks.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
 
