@@ -11,6 +11,7 @@
 #include <algorithm>
 
 #include "oc_internal.cuh"
+#include "ptx_sm100.cuh"
 
 namespace oc {
 namespace {
@@ -132,7 +133,8 @@ template <bool SMALLG>
 __global__ void __launch_bounds__(SWEEP_WARPS * 32)
 sweep_block_kernel(float* __restrict__ Wp, int64_t m, int64_t n, const float* __restrict__ U, int64_t j1, int G,
                    float maxq, int static_groups, const int32_t* __restrict__ perm, float* __restrict__ scales,
-                   float* __restrict__ zeros, unsigned char* __restrict__ codes8, float* __restrict__ Err) {
+                   float* __restrict__ zeros, unsigned char* __restrict__ codes8, float* __restrict__ Err,
+                   float* __restrict__ Err_lo) {
   extern __shared__ __align__(16) float Ub[];  // [SB][UPAD], skewed
   const int bw = static_cast<int>(::min((int64_t)SB, n - j1));
   {
@@ -253,9 +255,24 @@ sweep_block_kernel(float* __restrict__ Wp, int64_t m, int64_t n, const float* __
       pk.z = qv[8] | (qv[9] << 8) | (qv[10] << 16) | (qv[11] << 24);
       pk.w = qv[12] | (qv[13] << 8) | (qv[14] << 16) | (qv[15] << 24);
       *reinterpret_cast<uint4*>(codes8 + r * n + col0) = pk;
+      if (Err_lo) {
+        // the trailing product's operand, split for 3xTF32: hi = tf32(e), lo = tf32(e - hi)
 #pragma unroll
-      for (int i = 0; i < CPL; i += 4)
-        *reinterpret_cast<float4*>(Err + r * SB + CPL * q + i) = make_float4(ev[i], ev[i + 1], ev[i + 2], ev[i + 3]);
+        for (int i = 0; i < CPL; i += 4) {
+          float h[4], l[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            h[k] = tf32_rna(ev[i + k]);
+            l[k] = tf32_rna(ev[i + k] - h[k]);
+          }
+          *reinterpret_cast<float4*>(Err + r * SB + CPL * q + i) = make_float4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<float4*>(Err_lo + r * SB + CPL * q + i) = make_float4(l[0], l[1], l[2], l[3]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < CPL; i += 4)
+          *reinterpret_cast<float4*>(Err + r * SB + CPL * q + i) = make_float4(ev[i], ev[i + 1], ev[i + 2], ev[i + 3]);
+      }
     }
   }
 }
@@ -332,7 +349,7 @@ void launch_static_grid(const Ctx& c, const float* W, int64_t m, int64_t n, int 
 
 void launch_sweep_block(const Ctx& c, float* Wp, int64_t m, int64_t n, const float* U, int64_t j1, int G,
                         int wbits, bool static_groups, const int32_t* perm, float* scales, float* zeros,
-                        unsigned char* codes8, float* Err) {
+                        unsigned char* codes8, float* Err, float* Err_lo) {
   static bool attr_done[64] = {false};
   const int smem = (SB * UPAD + SB) * 4;
   if (!attr_done[c.device & 63]) {
@@ -349,11 +366,11 @@ void launch_sweep_block(const Ctx& c, float* Wp, int64_t m, int64_t n, const flo
   const bool small_g = !static_groups && G < CPL;
   if (small_g)
     sweep_block_kernel<true><<<grid, SWEEP_WARPS * 32, smem, c.stream>>>(Wp, m, n, U, j1, G, maxq, static_groups ? 1 : 0,
-                                                                          perm, scales, zeros, codes8, Err);
+                                                                          perm, scales, zeros, codes8, Err, Err_lo);
   else
     sweep_block_kernel<false><<<grid, SWEEP_WARPS * 32, smem, c.stream>>>(Wp, m, n, U, j1, G, maxq,
                                                                            static_groups ? 1 : 0, perm, scales, zeros,
-                                                                           codes8, Err);
+                                                                           codes8, Err, Err_lo);
   check_launch("sweep_block_kernel");
 }
 

@@ -224,14 +224,14 @@ void gptq_sweep_and_pack(const Ctx& c, float* Wp, int64_t m, int64_t n, const fl
     const int64_t bw = std::min<int64_t>(128, n - j1);
     const int64_t j2 = j1 + bw;
     {
+      // the sweep writes the block's errors already split for 3xTF32
       PhaseScope ps(c, kPhGptqSweep);
-      launch_sweep_block(c, Wp, m, n, U, j1, G, wbits, act_order, perm, scales, zeros, codes8, Err);
+      launch_sweep_block(c, Wp, m, n, U, j1, G, wbits, act_order, perm, scales, zeros, codes8, Errh, Errl);
     }
     if (j2 < n) {
       // W[:, j2:] -= Err U[j1:j2, j2:] on the tensor cores (3xTF32); B stored
       // = U^T[j2:, j1:j2] (rows j2.., columns j1..j1+bw of the transpose)
       PhaseScope ps(c, kPhGptqTrailing);
-      split_tf32(c, Err, m, bw, 128, Errh, Errl, 128);
       gemm_tf32x3(c, m, n - j2, bw, -1.f, Errh, Errl, 128, UTh + j2 * n + j1, UTl + j2 * n + j1, n, true, Wp + j2,
                   n, kANone);
     }

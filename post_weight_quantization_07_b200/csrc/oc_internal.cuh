@@ -182,7 +182,8 @@ void launch_static_grid(const Ctx& c, const float* W, int64_t m, int64_t n, int 
                         const unsigned char* dead, float* scales, float* zeros);
 void launch_sweep_block(const Ctx& c, float* Wp, int64_t m, int64_t n, const float* U,
                         int64_t j1, int G, int wbits, bool static_groups, const int32_t* perm,
-                        float* scales, float* zeros, unsigned char* codes8, float* Err);
+                        float* scales, float* zeros, unsigned char* codes8, float* Err,
+                        float* Err_lo = nullptr);
 // Packs codes8 (processing order) into the original-order bitstream; perm2
 // holds the processing order in its first n entries and receives the inverse
 // permutation in the next n.
