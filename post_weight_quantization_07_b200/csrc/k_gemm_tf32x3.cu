@@ -282,6 +282,273 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constan
   if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
+// ---------------------------------------------------------------- CTA-pair variant
+// Same product on clusters of two CTAs sharing each MMA (tcgen05 cta_group::2):
+// a pair owns a 256 x 256 tile of C; CTA r loads rows [128r, 128r + 128) of the
+// tile's A and of its B (hi and lo halves, 64 KB per 32-deep k slice) and
+// holds rows [128r, 128r + 128) of the accumulator (two 128 x 256 fp32
+// accumulators = all 512 TMEM columns).  Each SM thus loads the same bytes
+// per slice as the single-CTA kernel for twice the MMA work.  Both producers
+// arm the leader's "full" barrier with their own bytes; the leader issues
+// M=256 N=256 K=8 kind::tf32 MMAs (3 per k step) and commits to both CTAs.
+constexpr int PM = 256, PN = 256;              // pair tile
+constexpr int P_STAGES = 3;
+constexpr int P_STAGE_BYTES = 4 * TILE_BYTES;  // A_hi, A_lo, B_hi, B_lo (128 rows each)
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + EPI_BYTES + 1024 + 1024;
+static_assert(P_SMEM_BYTES <= 232448, "shared memory per CTA");
+constexpr uint32_t P_TMEM_COLS = 512;
+constexpr uint16_t kPairMask = 0x3;
+
+__device__ __forceinline__ bool pair_tile_skipped(const Params& p, int i0, int j0) {
+  return (p.flags & kCLowerOnly) && j0 > i0 + PM - 1;
+}
+
+__device__ __forceinline__ void pair_k_range(const Params& p, int i0, int j0, int& kb, int& ke) {
+  kb = 0;
+  ke = p.K;
+  if (p.flags & kAUpper) kb = max(kb, i0);
+  if (p.flags & kALower) ke = min(ke, i0 + PM);
+  if (p.flags & kBLower) kb = max(kb, j0);
+  if (p.flags & kBUpper) ke = min(ke, j0 + PN);
+  kb = (kb / BK) * BK;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_tf32x3_pair_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constant__ CUtensorMap mAl,
+                        const __grid_constant__ CUtensorMap mBh, const __grid_constant__ CUtensorMap mBl,
+                        const __grid_constant__ CUtensorMap mC, const Params p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* stage_base = smem;
+  unsigned char* epi_base = smem + P_STAGES * P_STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_base + EPI_BYTES);
+  uint64_t* full = bars;                   // leader: both CTAs' loads
+  uint64_t* empty = bars + P_STAGES;       // this CTA's ring slots
+  uint64_t* tfull = bars + 2 * P_STAGES;   // this CTA's accumulator half ready
+  uint64_t* tempty = tfull + 2;            // leader: both epilogues done
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  const int n_tiles = p.tiles_m * p.tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full[s], 2);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&mAh);
+    prefetch_tensormap(&mAl);
+    prefetch_tensormap(&mBh);
+    prefetch_tensormap(&mBl);
+    prefetch_tensormap(&mC);
+  }
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, P_TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int half = BM * static_cast<int>(rank);  // this CTA's rows of the pair tile
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer (both CTAs)
+    uint64_t issued = 0;
+    bool ok = true;
+    for (int t = cid; t < n_tiles && ok; t += ncl) {
+      const int i0 = (t % p.tiles_m) * PM, j0 = (t / p.tiles_m) * PN;
+      if (pair_tile_skipped(p, i0, j0)) continue;
+      int kb, ke;
+      pair_k_range(p, i0, j0, kb, ke);
+      for (int k0 = kb; k0 < ke; k0 += BK) {
+        const int s = static_cast<int>(issued % P_STAGES);
+        const uint32_t ph = static_cast<uint32_t>((issued / P_STAGES) & 1);
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&empty[s], ph ^ 1) && !*abort_flag;
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) { ok = false; break; }
+        if (lane == 0) {
+          unsigned char* st = stage_base + s * P_STAGE_BYTES;
+          mbar_arrive_expect_tx_cluster(mapa_shared(smem_u32(&full[s]), 0), P_STAGE_BYTES);
+          tma_load_2d_pair(&mAh, &full[s], st, k0, i0 + half);
+          tma_load_2d_pair(&mAl, &full[s], st + TILE_BYTES, k0, i0 + half);
+          tma_load_2d_pair(&mBh, &full[s], st + 2 * TILE_BYTES, k0, j0 + half);
+          tma_load_2d_pair(&mBl, &full[s], st + 3 * TILE_BYTES, k0, j0 + half);
+        }
+        __syncwarp();
+        ++issued;
+      }
+    }
+    if (lane == 0) {
+      if (!ok) {
+        record_error(p.status, kDevTimeout);
+        *abort_flag = 1;
+      }
+      if (leader) {
+        const uint64_t first = issued > P_STAGES ? issued - P_STAGES : 0;
+        for (uint64_t q = first; q < issued; ++q) {
+          if (!mbar_wait(&full[q % P_STAGES], static_cast<uint32_t>((q / P_STAGES) & 1))) {
+            record_error(p.status, kDevTimeout);
+            break;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (leader) {
+      // ---------------------------------------------------------------- MMA issuer (leader)
+      constexpr uint32_t idesc = instr_desc(2, 2, false, false, PM, PN);
+      uint64_t consumed = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = cid; t < n_tiles && ok; t += ncl) {
+        const int i0 = (t % p.tiles_m) * PM, j0 = (t / p.tiles_m) * PN;
+        if (pair_tile_skipped(p, i0, j0)) continue;
+        int kb, ke;
+        pair_k_range(p, i0, j0, kb, ke);
+        const int acc = it & 1;
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1));
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dcol = tmem_base + static_cast<uint32_t>(acc * PN);
+        for (int k0 = kb; k0 < ke; k0 += BK) {
+          const int s = static_cast<int>(consumed % P_STAGES);
+          const uint32_t ph = static_cast<uint32_t>((consumed / P_STAGES) & 1);
+          w = 1;
+          if (lane == 0) w = mbar_wait(&full[s], ph) && !*abort_flag;
+          w = __shfl_sync(0xffffffffu, w, 0);
+          if (!w) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sa = smem_u32(stage_base + s * P_STAGE_BYTES);
+            const uint32_t sah = sa, sal = sa + TILE_BYTES, sbh = sa + 2 * TILE_BYTES, sbl = sa + 3 * TILE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 8; ++kk) {
+              const uint64_t ah = smem_desc_sw128(sah + kk * 32, 16, 1024);
+              const uint64_t al = smem_desc_sw128(sal + kk * 32, 16, 1024);
+              const uint64_t bh = smem_desc_sw128(sbh + kk * 32, 16, 1024);
+              const uint64_t bl = smem_desc_sw128(sbl + kk * 32, 16, 1024);
+              const uint32_t first = (k0 == kb && kk == 0) ? 0u : 1u;
+              mma_tf32_ss_pair(dcol, al, bh, idesc, first);
+              mma_tf32_ss_pair(dcol, ah, bl, idesc, 1u);
+              mma_tf32_ss_pair(dcol, ah, bh, idesc, 1u);
+            }
+            mma_commit_pair(&empty[s], kPairMask);
+          }
+          __syncwarp();
+          ++consumed;
+        }
+        if (!ok) break;
+        if (lane == 0) mma_commit_pair(&tfull[acc], kPairMask);
+        __syncwarp();
+        ++it;
+      }
+      if (lane == 0) {
+        if (!ok) {
+          record_error(p.status, kDevTimeout);
+          *abort_flag = 1;
+        }
+        mma_commit_pair(drain, kPairMask);
+        if (!mbar_wait(drain, 0)) record_error(p.status, kDevTimeout);
+      }
+    } else {
+      if (lane == 0 && !mbar_wait(drain, 0)) record_error(p.status, kDevTimeout);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp - 4;
+    unsigned char* stage_buf = epi_base + q * 2 * EPI_BOX_BYTES;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    int it = 0, nbuf = 0;
+    bool ok = true;
+    for (int t = cid; t < n_tiles; t += ncl) {
+      const int i0 = (t % p.tiles_m) * PM, j0 = (t / p.tiles_m) * PN;
+      if (pair_tile_skipped(p, i0, j0)) continue;
+      int kb, ke;
+      pair_k_range(p, i0, j0, kb, ke);
+      const bool empty_k = kb >= ke;
+      const int acc = it & 1;
+      int w = 1;
+      if (lane == 0) w = mbar_wait(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1)) && !*abort_flag;
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (!w) { ok = false; break; }
+      tc_fence_after();
+      if (!(empty_k && p.accumulate)) {
+        for (int c = 0; c < PN / 32; ++c) {
+          uint32_t r[32];
+          if (!empty_k) {
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                   static_cast<uint32_t>(acc * PN + c * 32);
+            tmem_ld_32x32b_x32(taddr, r);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0u;
+          }
+          unsigned char* buf = stage_buf + (nbuf & 1) * EPI_BOX_BYTES;
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            float4 v;
+            v.x = __uint_as_float(r[4 * k + 0]) * p.alpha;
+            v.y = __uint_as_float(r[4 * k + 1]) * p.alpha;
+            v.z = __uint_as_float(r[4 * k + 2]) * p.alpha;
+            v.w = __uint_as_float(r[4 * k + 3]) * p.alpha;
+            *reinterpret_cast<float4*>(buf + lane * 128 + ((k ^ (lane & 7)) << 4)) = v;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (p.accumulate) tma_reduce_add_2d(&mC, buf, j0 + c * 32, i0 + half + 32 * q);
+            else tma_store_2d(&mC, buf, j0 + c * 32, i0 + half + 32 * q);
+            bulk_commit_group();
+          }
+          ++nbuf;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+      ++it;
+    }
+    if (!ok && lane == 0) {
+      record_error(p.status, kDevTimeout);
+      *abort_flag = 1;
+    }
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, P_TMEM_COLS);
+}
+
 // x_hi = tf32(x), x_lo = tf32(x - x_hi), both rounded to nearest (ties away).
 __device__ __forceinline__ float to_tf32(float x) {
   uint32_t r;
@@ -372,6 +639,44 @@ void gemm_tf32x3(const Ctx& c, int64_t M, int64_t N, int64_t K, float alpha, con
   p.alpha = alpha;
   p.accumulate = accumulate ? 1 : 0;
   p.status = c.status;
+  // A product with at least a wave of 256 x 256 tiles runs on CTA pairs (half
+  // the operand traffic per SM); smaller ones keep more, smaller tiles.
+  const int64_t pair_tiles = ((M + PM - 1) / PM) * ((N + PN - 1) / PN);
+  if (pair_tiles >= c.sm_count / 2) {
+    static int max_clusters[64] = {0};
+    const int dv = c.device & 63;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = P_SMEM_BYTES;
+    cfg.stream = c.stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (max_clusters[dv] == 0) {
+      check_cuda(cudaFuncSetAttribute(gemm_tf32x3_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      P_SMEM_BYTES),
+                 "cudaFuncSetAttribute(gemm_tf32x3_pair)");
+      cfg.gridDim = dim3(static_cast<unsigned>(2 * (c.sm_count / 2)), 1, 1);
+      int ncl = 0;
+      check_cuda(cudaOccupancyMaxActiveClusters(&ncl, gemm_tf32x3_pair_kernel, &cfg),
+                 "cudaOccupancyMaxActiveClusters(gemm_tf32x3_pair)");
+      if (ncl < 1) fail(OC_ERR_UNSUPPORTED, "gemm_tf32x3: no CTA pair fits on this device");
+      max_clusters[dv] = ncl;
+    }
+    Params q = p;
+    q.tiles_m = static_cast<int>((M + PM - 1) / PM);
+    q.tiles_n = static_cast<int>((N + PN - 1) / PN);
+    const int64_t clusters = std::min<int64_t>(pair_tiles, max_clusters[dv]);
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+    check_cuda(cudaLaunchKernelEx(&cfg, gemm_tf32x3_pair_kernel, mAh, mAl, mBh, mBl, mC, q),
+               "cudaLaunchKernelEx(gemm_tf32x3_pair)");
+    check_launch("gemm_tf32x3_pair_kernel");
+    return;
+  }
   const int64_t n_tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
   const int grid = static_cast<int>(std::min<int64_t>(n_tiles, c.sm_count));
   set_attr_once(c.device);
