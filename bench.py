@@ -537,6 +537,81 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- one layer over N GPUs
+
+def run_shard_layer(args, rank, world, local_rank):
+    """One layer split over the ranks: rank r takes token shard r (its share of
+    H and the cross term, all-reduced over NCCL) and row shard r of W (QEP and
+    GPTQ of those rows).  The whole job quantises one layer per step, so the
+    value is layers/s of the job (strong scaling)."""
+    import torch
+
+    import post_weight_quantization_07_b200 as oc
+    from post_weight_quantization_07_b200.sharded import quantize_layer_sharded, shard_range
+    from synthetic import CONFIGS, make_layer_device
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    spec = CONFIGS[args.workload]
+    if args.n_tok:
+        spec = spec.with_(n_tok=args.n_tok)
+    L = make_layer_device(spec, "cuda")  # the same layer on every rank
+    t0, t1 = shard_range(spec.n_tok, rank, world, align=64)
+    r0, r1 = shard_range(spec.d_out, rank, world)
+    X, Xh = L["X"][t0:t1].contiguous(), L["Xhat"][t0:t1].contiguous()
+    W = L["W"][r0:r1].contiguous()
+    del L
+    torch.cuda.empty_cache()
+    stream = torch.cuda.current_stream()
+    oc.oc_set_sync(False)
+    reduce = (lambda t: dist.all_reduce(t)) if dist is not None else (lambda t: None)
+
+    def step():
+        quantize_layer_sharded(W, X, Xh, spec.alpha, spec.damp, spec.wbits, spec.groupsize, spec.act_order,
+                               all_reduce=reduce)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    st = oc.oc_stream_status(stream)
+    if st != oc.OC_OK:
+        raise RuntimeError(f"sharded steps failed: {oc.oc_status_string(st)}")
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(args.steps / (ms / 1e3), 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16+f32",
+        "data": "synthetic",
+        "config": dict(workload_config(spec),
+                       parallelism=f"one layer over {world} rank(s): tokens and rows sharded, "
+                                   f"H and the cross term all-reduced"),
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- one 7B block
 
 BLOCK_GROUPS = ((0, 1, 2), (3,), (4, 5), (6,))  # q/k/v, o, gate/up, down of llama7b_layers()
@@ -664,6 +739,8 @@ def main():
                     help="calibration tokens per layer (default: the workload's own)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard-layer", action="store_true",
+                    help="one layer split over the ranks (tokens and rows) instead of one layer per rank")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -674,6 +751,8 @@ def main():
         run_reference(args, rank, world)
     elif args.workload == "c4_block":
         run_block(args, rank, world, local_rank)
+    elif args.shard_layer:
+        run_shard_layer(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

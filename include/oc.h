@@ -204,6 +204,32 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
                       float* zeros, int32_t* perm_out, void* stream);
 
 /*
+ * The layer's data-dependent terms over one shard of the calibration tokens:
+ *   H_part = 2 Xhat^T Xhat,   D_part = X^T Xhat - Xhat^T Xhat  (= (X - Xhat)^T Xhat)
+ * Both are sums over tokens, so the terms of a layer whose tokens are split
+ * over several GPUs are the element-wise sums of every shard's terms (one
+ * all-reduce); oc_quantize_from_terms then finishes the layer.  Same
+ * arithmetic as the first stages of oc_quantize_layer.
+ *   X, Xhat  bf16 [n_tok x n] (this shard);  n_tok >= 0 (0 gives zeros).
+ *   H_part, D_part  fp32 [n x n], overwritten.
+ */
+int oc_qep_terms(const void* X, const void* Xhat, int64_t n_tok, int64_t n, float* H_part, float* D_part,
+                 void* stream);
+
+/*
+ * oc_quantize_layer from the layer's global terms H = 2 Xhat^T Xhat and
+ * D = (X - Xhat)^T Xhat (e.g. all-reduced oc_qep_terms of the token shards):
+ * the QEP correction of W, then GPTQ of W_out with H.  Rows of W are
+ * independent in both steps, so a layer whose rows are split over GPUs runs
+ * this per shard of rows with the same H and D.
+ *   W, W_out  fp32 [m x n] (W_out must not alias W).   H, D fp32 [n x n], read only.
+ *   Other arguments and errors as oc_quantize_layer.
+ */
+int oc_quantize_from_terms(const float* W, int64_t m, int64_t n, const float* H, const float* D, float alpha,
+                           float damp, int wbits, int groupsize, int act_order, float* W_out, uint32_t* codes,
+                           float* scales, float* zeros, int32_t* perm_out, void* stream);
+
+/*
  * Dequantise packed GPTQ output: out[i][j] = scales[i][g] * (q[i][j] - zeros[i][g]),
  * g = j / groupsize, q read from row i's LSB-first bitstream of wbits-bit codes
  * (the layout oc_gptq_quantize writes).  This is the weight the quantised

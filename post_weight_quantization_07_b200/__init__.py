@@ -84,6 +84,10 @@ def _load():
     L.oc_quantize_layer_group.restype = i32
     L.oc_dequantize.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, i32, vp]
     L.oc_dequantize.restype = i32
+    L.oc_qep_terms.argtypes = [vp, vp, i64, i64, vp, vp, vp]
+    L.oc_qep_terms.restype = i32
+    L.oc_quantize_from_terms.argtypes = [vp, i64, i64, vp, vp, f32, f32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    L.oc_quantize_from_terms.restype = i32
     return L
 
 
@@ -362,3 +366,48 @@ def quantize_chain(Ws, X0, alpha, damp, wbits, groupsize, act_order, act="silu",
             y, yh = F.silu(y), F.silu(yh)
         x, xh = y.contiguous(), yh.contiguous()
     return layers, (x, xh)
+
+
+def oc_qep_terms(X, Xhat, H_part=None, D_part=None, stream=None):
+    """(2 Xhat^T Xhat, (X - Xhat)^T Xhat) over these tokens, fp32 [n x n] each."""
+    import torch
+    n_tok, n = Xhat.shape
+    if H_part is None:
+        H_part = torch.empty(n, n, dtype=torch.float32, device=Xhat.device)
+    if D_part is None:
+        D_part = torch.empty(n, n, dtype=torch.float32, device=Xhat.device)
+    xp = _dev_ptr(X, torch.bfloat16, "X", (n_tok, n)) if n_tok else None
+    hp = _dev_ptr(Xhat, torch.bfloat16, "Xhat", (n_tok, n)) if n_tok else None
+    st = _lib().oc_qep_terms(xp, hp, n_tok, n, _dev_ptr(H_part, torch.float32, "H_part", (n, n)),
+                             _dev_ptr(D_part, torch.float32, "D_part", (n, n)), _stream_handle(stream))
+    _check(st, "oc_qep_terms")
+    return H_part, D_part
+
+
+def oc_quantize_from_terms(W, H, D, alpha, damp, wbits, groupsize, act_order, W_out=None, codes=None,
+                           scales=None, zeros=None, perm_out=None, stream=None):
+    """QEP + GPTQ of W given the layer's global terms H and D.  Returns
+    (W_out, codes, scales, zeros, perm_out)."""
+    import torch
+    m, n = W.shape
+    G = n if groupsize == -1 else int(groupsize)
+    ng = max(1, n // G)
+    dev = W.device
+    if W_out is None:
+        W_out = torch.empty_like(W)
+    if codes is None:
+        codes = torch.empty(m, n * wbits // 32, dtype=torch.int32, device=dev)
+    if scales is None:
+        scales = torch.empty(m, ng, dtype=torch.float32, device=dev)
+    if zeros is None:
+        zeros = torch.empty(m, ng, dtype=torch.float32, device=dev)
+    pp = _dev_ptr(perm_out, torch.int32, "perm_out", (n,)) if perm_out is not None else None
+    st = _lib().oc_quantize_from_terms(
+        _dev_ptr(W, torch.float32, "W"), m, n, _dev_ptr(H, torch.float32, "H", (n, n)),
+        _dev_ptr(D, torch.float32, "D", (n, n)), float(alpha), float(damp), int(wbits), int(groupsize),
+        1 if act_order else 0, _dev_ptr(W_out, torch.float32, "W_out", (m, n)),
+        _dev_ptr(codes, torch.int32, "codes", (m, n * wbits // 32)),
+        _dev_ptr(scales, torch.float32, "scales", (m, ng)), _dev_ptr(zeros, torch.float32, "zeros", (m, ng)),
+        pp, _stream_handle(stream))
+    _check(st, "oc_quantize_from_terms")
+    return W_out, codes, scales, zeros, perm_out

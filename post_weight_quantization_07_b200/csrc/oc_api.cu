@@ -254,7 +254,11 @@ void gptq_sweep_and_pack(const Ctx& c, float* Wp, int64_t m, int64_t n, const fl
 int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n, const void* X, const void* Xhat,
                    int64_t n_tok, float alpha, float damp, int wbits, int groupsize, int act_order, float* H,
                    float* const* W_out, uint32_t* const* codes, float* const* scales, float* const* zeros,
-                   int32_t* perm_out, void* stream) {
+                   int32_t* perm_out, void* stream, const float* D_in = nullptr) {
+  // D_in non-null: H (read only) and D_in = d are the layer's global terms,
+  // already summed over all tokens (e.g. over the ranks of a token-sharded
+  // layer); X, Xhat and n_tok are then not used.
+  const bool terms_given = D_in != nullptr;
   if (count < 1 || count > kMaxGroup) fail(OC_ERR_INVALID_ARG, "count must be 1..%d", kMaxGroup);
   if (!W || !m || !W_out || !codes || !scales || !zeros) fail(OC_ERR_INVALID_ARG, "layer arrays must be non-null");
   int64_t m_max = 0;
@@ -266,10 +270,14 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
       if (W_out[l] == W[k]) fail(OC_ERR_INVALID_ARG, "W_out[%d] must not alias an input weight", l);
     m_max = std::max(m_max, m[l]);
   }
-  if (!X || !Xhat || !H) fail(OC_ERR_INVALID_ARG, "X, Xhat, H must be non-null");
-  if (n_tok < 1 || n_tok > (int64_t(1) << 31) - 64) fail(OC_ERR_INVALID_ARG, "n_tok out of range");
+  if (!H) fail(OC_ERR_INVALID_ARG, "H must be non-null");
+  if (!terms_given) {
+    if (!X || !Xhat) fail(OC_ERR_INVALID_ARG, "X, Xhat must be non-null");
+    if (n_tok < 1 || n_tok > (int64_t(1) << 31) - 64) fail(OC_ERR_INVALID_ARG, "n_tok out of range");
+    if (!aligned16(X) || !aligned16(Xhat)) fail(OC_ERR_INVALID_ARG, "X, Xhat must be 16-byte aligned");
+  }
   if (!(alpha == alpha) || alpha > 3.4e38f || alpha < -3.4e38f) fail(OC_ERR_INVALID_ARG, "alpha must be finite");
-  if (!aligned16(X) || !aligned16(Xhat) || !aligned16(H)) fail(OC_ERR_INVALID_ARG, "X, Xhat, H must be 16-byte aligned");
+  if (!aligned16(H)) fail(OC_ERR_INVALID_ARG, "H must be 16-byte aligned");
   const int64_t G = (groupsize == -1) ? n : groupsize;
   Ctx c = make_ctx(stream);
   const size_t nn = static_cast<size_t>(n) * n, mn = static_cast<size_t>(m_max) * n;
@@ -312,17 +320,19 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
   auto Gl = [&](int l) { return Gs + static_cast<size_t>(l) * mn; };
   const size_t nn_bytes = nn * sizeof(float);
 
-  {
-    PhaseScope ps(c, kPhHessianFix);
-    check_cuda(cudaMemsetAsync(H, 0, nn_bytes, c.stream), "memset H");
-  }
-  {
-    PhaseScope ps(c, kPhHessian);
-    launch_atb_bf16(c, Xhat, Xhat, n_tok, n, n, 2.0f, H, n, true);
-  }
-  {
-    PhaseScope ps(c, kPhHessianFix);
-    launch_mirror_upper(c, H, n);
+  if (!terms_given) {
+    {
+      PhaseScope ps(c, kPhHessianFix);
+      check_cuda(cudaMemsetAsync(H, 0, nn_bytes, c.stream), "memset H");
+    }
+    {
+      PhaseScope ps(c, kPhHessian);
+      launch_atb_bf16(c, Xhat, Xhat, n_tok, n, n, 2.0f, H, n, true);
+    }
+    {
+      PhaseScope ps(c, kPhHessianFix);
+      launch_mirror_upper(c, H, n);
+    }
   }
   // GPTQ's dampened Hessian equals QEP's 2A unless a column is dead (their
   // dampening constants then differ): one device-to-host read decides.
@@ -349,30 +359,34 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
     factor_inverse_upper(cs, UTh, UTl, Fs, UTh, n, true, fsplit);
     check_cuda(cudaEventRecord(ss.join, cs.stream), "cudaEventRecord(join)");
   }
-  {
-    PhaseScope ps(c, kPhQepCrossFix);
-    check_cuda(cudaMemsetAsync(D, 0, nn_bytes, c.stream), "memset d");
-  }
-  {
-    PhaseScope ps(c, kPhQepCross);
-    if (shared_factor) {
-      // In token ranges: between two launches the high-priority factorisation
-      // can take the freed SMs for its wide tensor-core products.
-      const int64_t parts = std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens));
-      const int64_t per = ((n_tok + parts - 1) / parts + 63) / 64 * 64;
-      const unsigned char* xb = static_cast<const unsigned char*>(X);
-      const unsigned char* hb = static_cast<const unsigned char*>(Xhat);
-      for (int64_t t0 = 0; t0 < n_tok; t0 += per) {
-        const int64_t len = std::min(per, n_tok - t0);
-        launch_atb_bf16(c, xb + t0 * n * 2, hb + t0 * n * 2, len, n, n, 1.0f, D, n, false, c.sm_count - kSideSMs);
-      }
-    } else {
-      launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false, 0);
+  if (terms_given) {
+    check_cuda(cudaMemcpyAsync(D, D_in, nn_bytes, cudaMemcpyDeviceToDevice, c.stream), "copy d");
+  } else {
+    {
+      PhaseScope ps(c, kPhQepCrossFix);
+      check_cuda(cudaMemsetAsync(D, 0, nn_bytes, c.stream), "memset d");
     }
-  }
-  {
-    PhaseScope ps(c, kPhQepCrossFix);
-    launch_sub_half(c, D, H, n);
+    {
+      PhaseScope ps(c, kPhQepCross);
+      if (shared_factor) {
+        // In token ranges: between two launches the high-priority factorisation
+        // can take the freed SMs for its wide tensor-core products.
+        const int64_t parts = std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens));
+        const int64_t per = ((n_tok + parts - 1) / parts + 63) / 64 * 64;
+        const unsigned char* xb = static_cast<const unsigned char*>(X);
+        const unsigned char* hb = static_cast<const unsigned char*>(Xhat);
+        for (int64_t t0 = 0; t0 < n_tok; t0 += per) {
+          const int64_t len = std::min(per, n_tok - t0);
+          launch_atb_bf16(c, xb + t0 * n * 2, hb + t0 * n * 2, len, n, n, 1.0f, D, n, false, c.sm_count - kSideSMs);
+        }
+      } else {
+        launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false, 0);
+      }
+    }
+    {
+      PhaseScope ps(c, kPhQepCrossFix);
+      launch_sub_half(c, D, H, n);
+    }
   }
   {
     // G = W d for every layer while the split copies of d^T are live
@@ -728,6 +742,54 @@ int oc_quantize_layer(const float* W, int64_t m, int64_t n, const void* X, const
   return guarded([&]() -> int {
     return quantize_group(1, &W, &m, n, X, Xhat, n_tok, alpha, damp, wbits, groupsize, act_order, H, &W_out, &codes,
                           &scales, &zeros, perm_out, stream);
+  });
+}
+
+int oc_qep_terms(const void* X, const void* Xhat, int64_t n_tok, int64_t n, float* H_part, float* D_part,
+                 void* stream) {
+  return guarded([&]() -> int {
+    if (!H_part || !D_part) fail(OC_ERR_INVALID_ARG, "H_part, D_part must be non-null");
+    if (n < 64 || n % 64) fail(OC_ERR_INVALID_ARG, "n must be a positive multiple of 64");
+    if (n_tok < 0 || n_tok > (int64_t(1) << 31) - 64) fail(OC_ERR_INVALID_ARG, "n_tok out of range");
+    if (n_tok > 0 && (!X || !Xhat)) fail(OC_ERR_INVALID_ARG, "X, Xhat must be non-null");
+    if ((n_tok > 0 && (!aligned16(X) || !aligned16(Xhat))) || !aligned16(H_part) || !aligned16(D_part))
+      fail(OC_ERR_INVALID_ARG, "X, Xhat, H_part, D_part must be 16-byte aligned");
+    Ctx c = make_ctx(stream);
+    const size_t nn_bytes = static_cast<size_t>(n) * n * sizeof(float);
+    {
+      PhaseScope ps(c, kPhHessianFix);
+      check_cuda(cudaMemsetAsync(H_part, 0, nn_bytes, c.stream), "memset H_part");
+      check_cuda(cudaMemsetAsync(D_part, 0, nn_bytes, c.stream), "memset D_part");
+    }
+    if (n_tok == 0) return finish(c);
+    {
+      PhaseScope ps(c, kPhHessian);
+      launch_atb_bf16(c, Xhat, Xhat, n_tok, n, n, 2.0f, H_part, n, true);
+    }
+    {
+      PhaseScope ps(c, kPhHessianFix);
+      launch_mirror_upper(c, H_part, n);
+    }
+    {
+      PhaseScope ps(c, kPhQepCross);
+      launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D_part, n, false);
+    }
+    {
+      PhaseScope ps(c, kPhQepCrossFix);
+      launch_sub_half(c, D_part, H_part, n);
+    }
+    return finish(c);
+  });
+}
+
+int oc_quantize_from_terms(const float* W, int64_t m, int64_t n, const float* H, const float* D, float alpha,
+                           float damp, int wbits, int groupsize, int act_order, float* W_out, uint32_t* codes,
+                           float* scales, float* zeros, int32_t* perm_out, void* stream) {
+  return guarded([&]() -> int {
+    if (!D) fail(OC_ERR_INVALID_ARG, "D must be non-null");
+    if (!aligned16(D)) fail(OC_ERR_INVALID_ARG, "D must be 16-byte aligned");
+    return quantize_group(1, &W, &m, n, nullptr, nullptr, 0, alpha, damp, wbits, groupsize, act_order,
+                          const_cast<float*>(H), &W_out, &codes, &scales, &zeros, perm_out, stream, D);
   });
 }
 

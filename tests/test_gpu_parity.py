@@ -445,3 +445,48 @@ def test_chain_qep_reduces_propagated_error_on_gpu():
         _, (x, xh) = oc.quantize_chain(Ws, dev(x0), alpha, 0.01, 3, 32, False)
         errs[alpha] = float((x.float() - xh.float()).norm() / x.float().norm())
     assert errs[0.5] < errs[0.0], errs
+
+
+# ----------------------------------------------------------------------------- sharded layers
+
+@pytest.mark.parametrize("act", [False, True])
+def test_token_and_row_shards_match_whole_layer(act):
+    # Two shards in one process: oc_qep_terms on each token half, their sum
+    # (what the all-reduce of a 2-GPU run computes), oc_quantize_from_terms on
+    # each half of the rows; against the oracle on the whole layer.
+    from post_weight_quantization_07_b200.sharded import shard_range
+    m, n, n_tok, wbits, G = 320, 512, 3000, 4, 128
+    L = random_layer_host(m, n, n_tok, seed=8200)
+    W64 = L["W"].astype(np.float64)
+    Ho = oracle.hessian(L["Xhat"])
+    Wpo = oracle.qep_correct(W64, L["X"], L["Xhat"], 0.5, 0.01, H=Ho)
+    ref = oracle.gptq_quantize(Wpo, Ho, wbits, G, 0.01, act)
+    Xd, Xhd, Wd = bf16_dev(L["X"]), bf16_dev(L["Xhat"]), dev(L["W"])
+    H = torch.zeros(n, n, device="cuda")
+    D = torch.zeros(n, n, device="cuda")
+    for r in range(2):
+        t0, t1 = shard_range(n_tok, r, 2, align=64)
+        Hp, Dp = oc.oc_qep_terms(Xd[t0:t1].contiguous(), Xhd[t0:t1].contiguous())
+        H += Hp
+        D += Dp
+    assert rel_fro(H.cpu().numpy(), Ho) <= H_TOL
+    perm = torch.empty(n, dtype=torch.int32, device="cuda")
+    for r in range(2):
+        r0, r1 = shard_range(m, r, 2)
+        Wp, codes, scales, zeros, _ = oc.oc_quantize_from_terms(Wd[r0:r1].contiguous(), H, D, 0.5, 0.01, wbits, G,
+                                                                act, perm_out=perm)
+        torch.cuda.synchronize()
+        assert np.abs(Wp.cpu().numpy() - Wpo[r0:r1]).max() <= QEP_TOL * np.abs(W64).max()
+        cg = oracle.unpack_codes(codes.cpu().numpy().view(np.uint32), wbits, n)
+        sg, zg = scales.cpu().numpy(), zeros.cpu().numpy()
+        st = oracle.teacher_forced_check(Wpo[r0:r1], Ho, wbits, G, 0.01, act, cg, sg, zg, perm=perm.cpu().numpy())
+        assert st["n_bad"] == 0 and st["zero_bad"] == 0 and st["scale_max_rel"] <= SCALE_TOL, (r, st)
+        ident = level_identity(cg, zg, ref["codes"][r0:r1], ref["zeros"][r0:r1], G)
+        assert ident >= code_frac_for(cg.size), (r, ident)
+
+
+def test_qep_terms_of_no_tokens_are_zero():
+    H, D = oc.oc_qep_terms(torch.empty(0, 128, dtype=torch.bfloat16, device="cuda"),
+                           torch.empty(0, 128, dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    assert float(H.abs().max()) == 0.0 and float(D.abs().max()) == 0.0
