@@ -228,6 +228,8 @@ def phase_work(spec, factorisations=1):
         "hessian_fixup": (8 * n * n, "byte", "hbm"),
         # clear d (4n^2), then d -= H/2 (read d and H, write d)
         "qep_cross_fixup": (16 * n * n, "byte", "hbm"),
+        # W (fp32), X and Xhat (bf16) read and written once each
+        "hadamard_rotate": (2 * (4 * m * n + 2 * 2 * N * n), "byte", "hbm"),
     }
 
 
@@ -332,8 +334,20 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     oc.oc_set_sync(False)
 
+    if args.rotate:
+        # rotation preprocessing: W, X and Xhat rotated by the same block
+        # Hadamard matrix every step, then the layer quantised in that basis
+        Wr, Xr, Xhr = torch.empty_like(W), torch.empty_like(X), torch.empty_like(Xh)
+
     def step():
-        oc.oc_quantize_layer(W, X, Xh, spec.alpha, spec.damp, spec.wbits, spec.groupsize,
+        if args.rotate:
+            oc.oc_hadamard_rotate(W, args.rotate, out=Wr, stream=stream)
+            oc.oc_hadamard_rotate(X, args.rotate, out=Xr, stream=stream)
+            oc.oc_hadamard_rotate(Xh, args.rotate, out=Xhr, stream=stream)
+            w_in, x_in, xh_in = Wr, Xr, Xhr
+        else:
+            w_in, x_in, xh_in = W, X, Xh
+        oc.oc_quantize_layer(w_in, x_in, xh_in, spec.alpha, spec.damp, spec.wbits, spec.groupsize,
                              spec.act_order, H=H, W_out=Wp, codes=codes, scales=scales,
                              zeros=zeros, stream=stream)
 
@@ -528,6 +542,9 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roof, "phases": phase_out, "gpu_launches": int(launches),
         "clocks": clocks, "e2e": e2e,
     }
+    if args.rotate:
+        line["config"]["rotation"] = (f"block-{args.rotate} Hadamard rotation of W, X and Xhat in every step "
+                                      f"(oc_hadamard_rotate), the layer quantised in the rotated basis")
     if world == 1 and not args.no_cpu_baseline:
         t_layer, t_meas = time_oracle_layer(spec)
         line["cpu_baseline"] = {"value": round(1.0 / t_layer, 6), "unit": UNIT,
@@ -739,6 +756,8 @@ def main():
                     help="calibration tokens per layer (default: the workload's own)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rotate", type=int, default=0, metavar="B",
+                    help="rotate W, X, Xhat by a block-B Hadamard matrix every step before quantising")
     ap.add_argument("--shard-layer", action="store_true",
                     help="one layer split over the ranks (tokens and rows) instead of one layer per rank")
     args = ap.parse_args()

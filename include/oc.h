@@ -230,6 +230,21 @@ int oc_quantize_from_terms(const float* W, int64_t m, int64_t n, const float* H,
                            float* scales, float* zeros, int32_t* perm_out, void* stream);
 
 /*
+ * Block Hadamard rotation along the features of each row:
+ *   Y = X (I_{n/block} (x) H_block) / sqrt(block),
+ * H_block the Sylvester Hadamard matrix (H_1 = [1], H_2k = [[H_k, H_k], [H_k, -H_k]]).
+ * The rotation is orthonormal and symmetric, so rotating a layer's weight
+ * rows (W H) and its input rows (X H, Xhat H) by the same matrix leaves its
+ * output W X^T unchanged while spreading outlier channels over their block
+ * before the Hessian is formed (OneComp release summary, section
+ * "進階預處理與後處理": rotation preprocessing with online Hadamard transforms).
+ *   X, Y    [rows x n] bf16 (bf16 = 1) or fp32 (bf16 = 0), row-major; Y may be X.
+ *   block   a power of two in 2..4096 dividing n.
+ * Sums in fp32, one rounding to the output type.
+ */
+int oc_hadamard_rotate(const void* X, int64_t rows, int64_t n, int block, void* Y, int bf16, void* stream);
+
+/*
  * Dequantise packed GPTQ output: out[i][j] = scales[i][g] * (q[i][j] - zeros[i][g]),
  * g = j / groupsize, q read from row i's LSB-first bitstream of wbits-bit codes
  * (the layout oc_gptq_quantize writes).  This is the weight the quantised

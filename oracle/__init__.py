@@ -546,3 +546,27 @@ def quantize_chain(Ws, x0, alpha: float, damp: float, wbits: int, groupsize: int
         x = _bf16(_act(_bf16(x @ _bf16(W).T), act))
         xh = _bf16(_act(_bf16(xh @ _bf16(q["deq"]).T), act))
     return layers, (x, xh)
+
+
+# ----------------------------------------------------------------------------- Hadamard rotation
+
+def hadamard(b: int):
+    """Sylvester Hadamard matrix of order b (a power of two): H_1 = [1],
+    H_2k = [[H_k, H_k], [H_k, -H_k]]."""
+    if b < 1 or b & (b - 1):
+        raise ValueError("b must be a power of two")
+    H = np.ones((1, 1))
+    while H.shape[0] < b:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def hadamard_rotate(x, b: int):
+    """x (I (x) H_b) / sqrt(b) along the last axis (rotation preprocessing,
+    OneComp release summary section "進階預處理與後處理")."""
+    x = _f64(x)
+    n = x.shape[-1]
+    if n % b:
+        raise ValueError("b must divide the last axis")
+    Hb = hadamard(b) / np.sqrt(b)
+    return (x.reshape(-1, n // b, b) @ Hb).reshape(x.shape)

@@ -88,6 +88,8 @@ def _load():
     L.oc_qep_terms.restype = i32
     L.oc_quantize_from_terms.argtypes = [vp, i64, i64, vp, vp, f32, f32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
     L.oc_quantize_from_terms.restype = i32
+    L.oc_hadamard_rotate.argtypes = [vp, i64, i64, i32, vp, i32, vp]
+    L.oc_hadamard_rotate.restype = i32
     return L
 
 
@@ -411,3 +413,19 @@ def oc_quantize_from_terms(W, H, D, alpha, damp, wbits, groupsize, act_order, W_
         pp, _stream_handle(stream))
     _check(st, "oc_quantize_from_terms")
     return W_out, codes, scales, zeros, perm_out
+
+
+def oc_hadamard_rotate(X, block, out=None, stream=None):
+    """X (I (x) H_block) / sqrt(block) along the last axis of a 2-D bf16 or fp32
+    tensor (out may be X)."""
+    import torch
+    rows, n = X.shape
+    if X.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("X must be bf16 or fp32")
+    if out is None:
+        out = torch.empty_like(X)
+    st = _lib().oc_hadamard_rotate(_dev_ptr(X, X.dtype, "X", (rows, n)) if rows else None, rows, n, int(block),
+                                   _dev_ptr(out, X.dtype, "out", (rows, n)) if rows else None,
+                                   1 if X.dtype == torch.bfloat16 else 0, _stream_handle(stream))
+    _check(st, "oc_hadamard_rotate")
+    return out

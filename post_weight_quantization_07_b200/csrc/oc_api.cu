@@ -720,6 +720,26 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
   });
 }
 
+int oc_hadamard_rotate(const void* X, int64_t rows, int64_t n, int block, void* Y, int bf16, void* stream) {
+  return guarded([&]() -> int {
+    if (rows < 0 || n < 1) fail(OC_ERR_INVALID_ARG, "rows must be >= 0 and n >= 1");
+    if (rows == 0) return OC_OK;
+    if (!X || !Y) fail(OC_ERR_INVALID_ARG, "X and Y must be non-null");
+    if (block < 2 || block > 4096 || (block & (block - 1))) fail(OC_ERR_INVALID_ARG, "block must be a power of two in 2..4096");
+    if (n % block) fail(OC_ERR_INVALID_ARG, "block must divide n");
+    if (bf16 != 0 && bf16 != 1) fail(OC_ERR_INVALID_ARG, "bf16 must be 0 or 1");
+    if (!aligned16(X) || !aligned16(Y)) fail(OC_ERR_INVALID_ARG, "X and Y must be 16-byte aligned");
+    int log2b = 0;
+    while ((1 << log2b) < block) ++log2b;
+    Ctx c = make_ctx(stream);
+    {
+      PhaseScope ps(c, kPhRotate);
+      launch_hadamard(c, X, Y, rows, n, log2b, bf16 != 0);
+    }
+    return finish(c);
+  });
+}
+
 int oc_dequantize(const uint32_t* codes, const float* scales, const float* zeros, int64_t m, int64_t n, int wbits,
                   int groupsize, void* out, int out_bf16, void* stream) {
   return guarded([&]() -> int {

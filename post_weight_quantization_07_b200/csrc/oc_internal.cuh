@@ -56,6 +56,7 @@ enum Phase : int {
   kPhGptqPack,      // inverse permutation + bit packing
   kPhHessianFix,    // clearing H, mirroring its upper triangle
   kPhQepCrossFix,   // clearing d, subtracting Xhat^T Xhat
+  kPhRotate,        // Hadamard rotation
   kNumPhases
 };
 
@@ -187,6 +188,8 @@ void launch_sweep_block(const Ctx& c, float* Wp, int64_t m, int64_t n, const flo
 // Packs codes8 (processing order) into the original-order bitstream; perm2
 // holds the processing order in its first n entries and receives the inverse
 // permutation in the next n.
+// Y = X (I (x) H_b) / sqrt(b) along rows of n features, b = 2^log2b <= 4096.
+void launch_hadamard(const Ctx& c, const void* X, void* Y, int64_t rows, int64_t n, int log2b, bool bf16);
 // out[i][j] = scale * (code - zero), fp32 or bf16, original column order.
 void launch_dequant(const Ctx& c, const uint32_t* codes, const float* scales, const float* zeros, int64_t m,
                     int64_t n, int wbits, int64_t G, void* out, bool bf16);

@@ -490,3 +490,40 @@ def test_qep_terms_of_no_tokens_are_zero():
                            torch.empty(0, 128, dtype=torch.bfloat16, device="cuda"))
     torch.cuda.synchronize()
     assert float(H.abs().max()) == 0.0 and float(D.abs().max()) == 0.0
+
+
+# ----------------------------------------------------------------------------- Hadamard rotation
+
+@pytest.mark.parametrize("rows,n,block", [(3, 4096, 4096), (5, 4096, 2048), (7, 11008, 256), (4, 1536, 512),
+                                          (9, 96, 32), (33, 64, 2), (2, 8192, 16)])
+def test_hadamard_rotation_matches_oracle(rows, n, block):
+    rng = np.random.default_rng(rows * 1000 + block)
+    x = rng.standard_normal((rows, n)).astype(np.float32)
+    x[:, :3] *= 20.0
+    want = oracle.hadamard_rotate(x, block)
+    y32 = oc.oc_hadamard_rotate(dev(x), block)
+    torch.cuda.synchronize()
+    # fp32: log2(block) rounded butterfly stages and one scaling, each adding
+    # at most a few ulps of the (orthonormally bounded) magnitudes
+    tol = 4e-7 * (np.log2(block) + 1) * np.abs(x).max()
+    assert np.abs(y32.cpu().numpy() - want).max() <= tol
+    xb = oracle._bf16(x)
+    yb = oc.oc_hadamard_rotate(bf16_dev(xb), block)
+    torch.cuda.synchronize()
+    wantb = oracle.hadamard_rotate(xb, block)
+    got = yb.float().cpu().numpy()
+    # one rounding to bf16 of a value within fp32 error of the exact rotation
+    assert np.mean(got == oracle._bf16(wantb)) >= 0.99
+    assert np.abs(got - wantb).max() <= 2.0 ** -8 * np.abs(wantb).max()
+
+
+def test_hadamard_rotation_in_place_and_layer_output_invariance():
+    rng = np.random.default_rng(95)
+    W = dev(rng.standard_normal((64, 4096)).astype(np.float32))
+    X = dev(rng.standard_normal((300, 4096)).astype(np.float32))
+    ref = W @ X.t()
+    Wr = oc.oc_hadamard_rotate(W, 4096)
+    oc.oc_hadamard_rotate(X, 4096, out=X)   # in place
+    torch.cuda.synchronize()
+    got = Wr.double() @ X.double().t()
+    assert float((got - ref.double()).abs().max()) <= 1e-3 * float(ref.abs().max())

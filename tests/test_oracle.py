@@ -438,3 +438,23 @@ def test_chain_qep_reduces_propagated_error():
         _, (x, xh) = oracle.quantize_chain(Ws, x0, alpha, 0.01, 3, 16, False)
         errs[alpha] = np.linalg.norm(x - xh) / np.linalg.norm(x)
     assert errs[0.5] < errs[0.0] and errs[1.0] < errs[0.0], errs
+
+
+def test_hadamard_is_sylvester_and_orthogonal():
+    import scipy.linalg as sla
+    for b in (1, 2, 8, 64):
+        H = oracle.hadamard(b)
+        assert np.array_equal(H, sla.hadamard(b))
+        assert np.array_equal(H @ H.T, b * np.eye(b))
+
+
+def test_hadamard_rotation_preserves_layer_output_and_is_an_involution():
+    rng = np.random.default_rng(76)
+    W = rng.standard_normal((5, 96))
+    X = rng.standard_normal((40, 96))
+    for b in (2, 32):
+        Wr, Xr = oracle.hadamard_rotate(W, b), oracle.hadamard_rotate(X, b)
+        assert np.allclose(Wr @ Xr.T, W @ X.T, rtol=0, atol=1e-12)
+        assert np.allclose(oracle.hadamard_rotate(Xr, b), X, rtol=0, atol=1e-12)
+        # blocks act independently: the first block of a row only mixes its own b features
+        assert np.allclose(Xr[:, :b], X[:, :b] @ (oracle.hadamard(b) / np.sqrt(b)), rtol=0, atol=1e-12)
