@@ -218,7 +218,7 @@ void check_gptq_args(const float* W, int64_t m, int64_t n, int wbits, int groups
 // tensor-core trailing updates, then packing (and the processing order out).
 void gptq_sweep_and_pack(const Ctx& c, float* Wp, int64_t m, int64_t n, const float* U, const float* UTh,
                          const float* UTl, int G, int wbits, bool act_order, int32_t* perm, float* scales,
-                         float* zeros, unsigned char* codes8, float* Err, float* Errh, float* Errl, uint32_t* codes,
+                         float* zeros, unsigned char* codes8, float* Errh, float* Errl, uint32_t* codes,
                          int32_t* perm_out) {
   for (int64_t j1 = 0; j1 < n; j1 += 128) {
     const int64_t bw = std::min<int64_t>(128, n - j1);
@@ -293,7 +293,7 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
   sizing.take<float>(mn * count);         // G -> T, one per layer
   sizing.take<float>(mn);                 // permuted working copy of W
   sizing.take<unsigned char>(mn);         // codes, processing order
-  sizing.take<float>(3 * static_cast<size_t>(m_max) * 128);  // block errors and their halves
+  sizing.take<float>(2 * static_cast<size_t>(m_max) * 128);  // block errors, hi and lo halves
   sizing.take<int32_t>(2 * static_cast<size_t>(n));          // order | inverse
   sizing.take<unsigned char>(n);          // dead-column mask
   sizing.take<float>(factor_split_floats(n));
@@ -310,8 +310,7 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
   float* Gs = cv.take<float>(mn * count);
   float* Wp = cv.take<float>(mn);
   unsigned char* codes8 = cv.take<unsigned char>(mn);
-  float* Err = cv.take<float>(3 * static_cast<size_t>(m_max) * 128);
-  float* Errh = Err + static_cast<size_t>(m_max) * 128;
+  float* Errh = cv.take<float>(2 * static_cast<size_t>(m_max) * 128);
   float* Errl = Errh + static_cast<size_t>(m_max) * 128;
   int32_t* perm = cv.take<int32_t>(2 * static_cast<size_t>(n));
   unsigned char* dead = cv.take<unsigned char>(n);
@@ -438,7 +437,7 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
         if (act_order) launch_static_grid(c, W_out[l], m[l], n, static_cast<int>(G), wbits, dead, scales[l], zeros[l]);
       }
       gptq_sweep_and_pack(c, Wp, m[l], n, D, UTh, UTl, static_cast<int>(G), wbits, act_order != 0, perm, scales[l],
-                          zeros[l], codes8, Err, Errh, Errl, codes[l], l == 0 ? perm_out : nullptr);
+                          zeros[l], codes8, Errh, Errl, codes[l], l == 0 ? perm_out : nullptr);
     }
     return finish(c);
   }
@@ -468,7 +467,7 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
       launch_static_grid(c, W_out[l], m[l], n, static_cast<int>(G), wbits, dead, scales[l], zeros[l]);
     }
     gptq_sweep_and_pack(c, Wp, m[l], n, D, UTh, UTl, static_cast<int>(G), wbits, act_order != 0, perm, scales[l],
-                        zeros[l], codes8, Err, Errh, Errl, codes[l], l == 0 ? perm_out : nullptr);
+                        zeros[l], codes8, Errh, Errl, codes[l], l == 0 ? perm_out : nullptr);
   }
   return finish(c);
 }
@@ -676,7 +675,6 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
     sizing.take<float>(nn + 4096);     // recursion scratch -> U_lo
     sizing.take<float>(mn);            // Wp
     sizing.take<unsigned char>(mn);    // codes8
-    sizing.take<float>(static_cast<size_t>(m) * 128);  // Err
     sizing.take<float>(static_cast<size_t>(m) * 128);  // Err_hi
     sizing.take<float>(static_cast<size_t>(m) * 128);  // Err_lo
     sizing.take<int32_t>(2 * static_cast<size_t>(n));  // perm | inverse
@@ -689,7 +687,6 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
     float* scratch = cv.take<float>(nn + 4096);
     float* Wp = cv.take<float>(mn);
     unsigned char* codes8 = cv.take<unsigned char>(mn);
-    float* Err = cv.take<float>(static_cast<size_t>(m) * 128);
     float* Errh = cv.take<float>(static_cast<size_t>(m) * 128);
     float* Errl = cv.take<float>(static_cast<size_t>(m) * 128);
     int32_t* perm = cv.take<int32_t>(2 * static_cast<size_t>(n));
@@ -715,7 +712,7 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
       if (act_order) launch_static_grid(c, W, m, n, static_cast<int>(G), wbits, dead, scales, zeros);
     }
     gptq_sweep_and_pack(c, Wp, m, n, U, UTh, UTl, static_cast<int>(G), wbits, act_order != 0, perm, scales, zeros,
-                        codes8, Err, Errh, Errl, codes, perm_out);
+                        codes8, Errh, Errl, codes, perm_out);
     return finish(c);
   });
 }
