@@ -589,6 +589,7 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
     sizing.take<float>(mn);                       // W_hi -> G_hi -> T_hi
     sizing.take<float>(mn);                       // W_lo -> G_lo -> T_lo
     sizing.take<float>(mn);                       // G -> T
+    sizing.take<float>(nn + 4096);                // recursion scratch of the side-stream factorisation
     sizing.take<float>(factor_split_floats(n));   // split copies inside the factorisation
     sizing.take<DiagStats>(1);
     Carve cv{workspace(c, sizing.off + 256)};
@@ -601,6 +602,7 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
     float* Ph = cv.take<float>(mn);
     float* Pl = cv.take<float>(mn);
     float* G = cv.take<float>(mn);
+    float* Fs = cv.take<float>(nn + 4096);
     float* fsplit = cv.take<float>(factor_split_floats(n));
     DiagStats* stats = cv.take<DiagStats>(1);
 
@@ -613,13 +615,37 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
       launch_mirror_upper(c, Hs, n);
       Hp = Hs;
     }
+    // 2A = Hp + damp mean(diag Hp) I = R R^T;  U = R^-1 upper, A^-1 = 2 U^T U.
+    // The factorisation needs only H: it runs on the high-priority side stream
+    // (into UTh, with UTl and Fs as scratch) beside the cross product, which
+    // runs in token ranges so that the factorisation's wide products can take
+    // SMs between its launches.
+    SideStream& ss = side_stream(c.device);
+    Ctx cs = c;
+    cs.stream = ss.stream;
+    check_cuda(cudaEventRecord(ss.fork, c.stream), "cudaEventRecord(fork)");
+    check_cuda(cudaStreamWaitEvent(cs.stream, ss.fork, 0), "cudaStreamWaitEvent(fork)");
+    {
+      PhaseScope ps(cs, kPhFactor);
+      launch_diag_stats(cs, Hp, n, damp, 1.0f, false, stats, nullptr);
+      launch_build_reversed(cs, Hp, n, nullptr, stats, 1.0f, false, UTh);
+      factor_inverse_upper(cs, UTh, UTl, Fs, UTh, n, true, fsplit);
+    }
+    check_cuda(cudaEventRecord(ss.join, cs.stream), "cudaEventRecord(join)");
     {
       PhaseScope ps(c, kPhQepCrossFix);
       check_cuda(cudaMemsetAsync(D, 0, nn * sizeof(float), c.stream), "memset D");
     }
     {
       PhaseScope ps(c, kPhQepCross);
-      launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false);
+      const int64_t parts = std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens));
+      const int64_t per = ((n_tok + parts - 1) / parts + 63) / 64 * 64;
+      const unsigned char* xb = static_cast<const unsigned char*>(X);
+      const unsigned char* hb = static_cast<const unsigned char*>(Xhat);
+      for (int64_t t0 = 0; t0 < n_tok; t0 += per) {
+        const int64_t len = std::min(per, n_tok - t0);
+        launch_atb_bf16(c, xb + t0 * n * 2, hb + t0 * n * 2, len, n, n, 1.0f, D, n, false, c.sm_count - kSideSMs);
+      }
     }
     {
       PhaseScope ps(c, kPhQepCrossFix);
@@ -632,16 +658,11 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
       split_tf32(c, W, m, n, n, Ph, Pl, n);
       gemm_tf32x3(c, m, n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, G, n, kANone);
     }
-    {
-      // 2A = Hp + damp mean(diag Hp) I = R R^T;  U = R^-1 upper, A^-1 = 2 U^T U
-      PhaseScope ps(c, kPhFactor);
-      launch_diag_stats(c, Hp, n, damp, 1.0f, false, stats, nullptr);
-      launch_build_reversed(c, Hp, n, nullptr, stats, 1.0f, false, D);
-      factor_inverse_upper(c, D, Xi, scratch, D, n, true, fsplit);
-    }
+    check_cuda(cudaStreamWaitEvent(c.stream, ss.join, 0), "cudaStreamWaitEvent(join)");
     {
       // W_out = W + alpha G A^-1 = W + 2 alpha (G U^T) U
       PhaseScope ps(c, kPhQepApply);
+      check_cuda(cudaMemcpyAsync(D, UTh, nn * sizeof(float), cudaMemcpyDeviceToDevice, c.stream), "copy U");
       const float* U = D;
       float* Uh = Xi;
       float* Ul = scratch;
