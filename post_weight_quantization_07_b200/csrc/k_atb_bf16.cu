@@ -10,15 +10,19 @@
 // (tcgen05 cta_group::2).  A pair owns a 256 x 256 output tile: CTA r holds
 // features [128r, 128r + 128) of the tile's A columns and of its B columns in
 // its shared memory and rows [128r, 128r + 128) of the fp32 accumulator in its
-// TMEM, so each SM loads 32 KB per 64-token stage for a 128 x 256 x 64 share
-// of the MMA work (a lone CTA would need 48 KB).  256 threads per CTA:
-//   warp 0       TMA producer: 2 + 2 boxes of 64 features x 64 tokens per
-//                stage, 128-byte swizzle, 6-stage ring; both CTAs' bytes are
+// TMEM, so each SM loads 64 KB per 128-token stage for a 128 x 256 x 128 share
+// of the MMA work (a lone CTA would need 96 KB).  256 threads per CTA:
+//   warp 0       TMA producer: 2 + 2 boxes of 64 features x 128 tokens per
+//                stage, 128-byte swizzle, 3-stage ring; both CTAs' bytes are
 //                counted on the leader's "full" barrier, which each producer
-//                arms with its own 32 KB.
+//                arms with its own 64 KB.  Long stages matter more than a deep
+//                ring here: each stage costs a fixed handshake (barrier waits,
+//                TMA issue, commit), and with the same 192 KB in flight,
+//                32-, 64- and 128-token stages ran at about 0.39, 0.56 and
+//                0.65 TFLOP/s per MHz.
 //   warp 1       TMEM owner (both CTAs allocate 512 columns together = two
 //                accumulators) and, in the leader CTA only, MMA issuer:
-//                M=256 N=256 K=16, four per stage, committed to the stage's
+//                M=256 N=256 K=16, eight per stage, committed to the stage's
 //                "empty" barrier in both CTAs; a unit's last commit signals
 //                both CTAs' epilogues.
 //   warps 4..7   epilogue (both CTAs): tcgen05.ld 32 lanes x 32 columns, scale,
@@ -43,12 +47,12 @@ constexpr int TM = 256;          // pair tile rows (A features)
 constexpr int TN = 256;          // pair tile cols (B features) = TMEM columns per accumulator
 constexpr int HM = TM / 2;       // rows per CTA = TMEM lanes
 constexpr int HN = TN / 2;       // B features held per CTA
-constexpr int BK = 64;           // tokens per stage
-constexpr int STAGES = 6;
-constexpr int A_BYTES = HM * BK * 2;              // 16 KB
-constexpr int B_BYTES = HN * BK * 2;              // 16 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 32 KB per CTA
-constexpr int BOX_BYTES = 64 * BK * 2;            // one 64-feature x 64-token box, 8 KB
+constexpr int BK = 128;          // tokens per stage
+constexpr int STAGES = 3;
+constexpr int A_BYTES = HM * BK * 2;              // 32 KB
+constexpr int B_BYTES = HN * BK * 2;              // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 64 KB per CTA
+constexpr int BOX_BYTES = 64 * BK * 2;            // one 64-feature x 128-token box, 16 KB
 constexpr int EPI_WARPS = 4;
 constexpr int EPI_BOX_BYTES = 32 * 32 * 4;        // 32x32 fp32 staging box
 constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BOX_BYTES;
@@ -388,7 +392,7 @@ void launch_atb_bf16(const Ctx& c, const void* A, const void* B, int64_t n_tok, 
   // units (about four per cluster) to balance the clusters.
   const int64_t want_chunks = std::max<int64_t>(1, (4 * clusters_avail + p.n_tiles - 1) / p.n_tiles);
   int64_t kcs = (stages_total + want_chunks - 1) / want_chunks;
-  kcs = std::max<int64_t>(16, std::min<int64_t>(128, kcs));
+  kcs = std::max<int64_t>(1024 / BK, std::min<int64_t>(8192 / BK, kcs));
   kcs = std::min(kcs, stages_total);
   p.kc_stages = static_cast<int>(kcs);
   p.n_kc = static_cast<int>((stages_total + kcs - 1) / kcs);
