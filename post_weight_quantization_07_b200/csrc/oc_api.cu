@@ -362,8 +362,9 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
     check_cuda(cudaMemcpyAsync(D, D_in, nn_bytes, cudaMemcpyDeviceToDevice, c.stream), "copy d");
   } else {
     {
+      // d = X^T Xhat - Xhat^T Xhat: start from -H/2 and add the cross product
       PhaseScope ps(c, kPhQepCrossFix);
-      check_cuda(cudaMemsetAsync(D, 0, nn_bytes, c.stream), "memset d");
+      launch_neg_half(c, H, D, n);
     }
     {
       PhaseScope ps(c, kPhQepCross);
@@ -381,10 +382,6 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
       } else {
         launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false, 0);
       }
-    }
-    {
-      PhaseScope ps(c, kPhQepCrossFix);
-      launch_sub_half(c, D, H, n);
     }
   }
   {
@@ -634,7 +631,7 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
     check_cuda(cudaEventRecord(ss.join, cs.stream), "cudaEventRecord(join)");
     {
       PhaseScope ps(c, kPhQepCrossFix);
-      check_cuda(cudaMemsetAsync(D, 0, nn * sizeof(float), c.stream), "memset D");
+      launch_neg_half(c, Hp, D, n);
     }
     {
       PhaseScope ps(c, kPhQepCross);
@@ -646,10 +643,6 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
         const int64_t len = std::min(per, n_tok - t0);
         launch_atb_bf16(c, xb + t0 * n * 2, hb + t0 * n * 2, len, n, n, 1.0f, D, n, false, c.sm_count - kSideSMs);
       }
-    }
-    {
-      PhaseScope ps(c, kPhQepCrossFix);
-      launch_sub_half(c, D, Hp, n);
     }
     {
       // G = W d on the tensor cores (3xTF32 from split operands)
@@ -797,7 +790,7 @@ int oc_qep_terms(const void* X, const void* Xhat, int64_t n_tok, int64_t n, floa
     {
       PhaseScope ps(c, kPhHessianFix);
       check_cuda(cudaMemsetAsync(H_part, 0, nn_bytes, c.stream), "memset H_part");
-      check_cuda(cudaMemsetAsync(D_part, 0, nn_bytes, c.stream), "memset D_part");
+      if (n_tok == 0) check_cuda(cudaMemsetAsync(D_part, 0, nn_bytes, c.stream), "memset D_part");
     }
     if (n_tok == 0) return finish(c);
     {
@@ -809,12 +802,12 @@ int oc_qep_terms(const void* X, const void* Xhat, int64_t n_tok, int64_t n, floa
       launch_mirror_upper(c, H_part, n);
     }
     {
-      PhaseScope ps(c, kPhQepCross);
-      launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D_part, n, false);
+      PhaseScope ps(c, kPhQepCrossFix);
+      launch_neg_half(c, H_part, D_part, n);
     }
     {
-      PhaseScope ps(c, kPhQepCrossFix);
-      launch_sub_half(c, D_part, H_part, n);
+      PhaseScope ps(c, kPhQepCross);
+      launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D_part, n, false);
     }
     return finish(c);
   });

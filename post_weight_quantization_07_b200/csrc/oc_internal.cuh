@@ -200,7 +200,7 @@ void launch_pack(const Ctx& c, const unsigned char* codes8, int64_t m, int64_t n
 void launch_invert_perm(const Ctx& c, int32_t* perm2, int64_t n);
 
 // QEP pieces.
-void launch_sub_half(const Ctx& c, float* D, const float* H, int64_t n);  // D -= H/2
+void launch_neg_half(const Ctx& c, const float* H, float* D, int64_t n);  // D = -H/2
 void launch_copy_f32(const Ctx& c, const float* src, float* dst, int64_t count);
 void launch_fill_f32(const Ctx& c, float* dst, int64_t count, float v);
 void launch_check_finite(const Ctx& c, const float* x, int64_t count);
