@@ -591,6 +591,76 @@ __global__ void split_tf32_t_kernel(const float* __restrict__ src, int64_t rows,
   }
 }
 
+// Vectorised split of a matrix whose rows are 16-byte aligned and a multiple
+// of 4 floats long: 4 independent float4 per thread in flight, grid-stride.
+__device__ __forceinline__ void split4(const float4 x, float4& h, float4& l) {
+  h = make_float4(to_tf32(x.x), to_tf32(x.y), to_tf32(x.z), to_tf32(x.w));
+  l = make_float4(to_tf32(x.x - h.x), to_tf32(x.y - h.y), to_tf32(x.z - h.z), to_tf32(x.w - h.w));
+}
+
+__global__ void __launch_bounds__(256) split_tf32_v4_kernel(const float4* __restrict__ src, int64_t rows,
+                                                            int64_t cols4, int64_t lds4, float4* __restrict__ hi,
+                                                            float4* __restrict__ lo, int64_t ldd4) {
+  const int64_t total = rows * cols4;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t e0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e0 < total; e0 += 4 * stride) {
+    float4 x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t e = e0 + u * stride;
+      if (e < total) x[u] = src[(e / cols4) * lds4 + e % cols4];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t e = e0 + u * stride;
+      if (e < total) {
+        float4 h, l;
+        split4(x[u], h, l);
+        const int64_t d = (e / cols4) * ldd4 + e % cols4;
+        hi[d] = h;
+        lo[d] = l;
+      }
+    }
+  }
+}
+
+// Vectorised transposing split through 64 x 64 tiles (rows and cols multiples
+// of 4, 16-byte aligned rows): float4 reads along the source rows, float4
+// writes along the destination rows.
+constexpr int TT = 64;
+__global__ void __launch_bounds__(256) split_tf32_t64_kernel(const float* __restrict__ src, int64_t rows,
+                                                             int64_t cols, int64_t lds, float* __restrict__ hi,
+                                                             float* __restrict__ lo, int64_t ldd) {
+  __shared__ float t[TT][TT + 1];
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * TT, c0 = static_cast<int64_t>(blockIdx.x) * TT;
+  const int tid = threadIdx.x;
+  const int cq = tid & 15, rq = tid >> 4;  // 16 float4 columns x 16 rows per pass
+#pragma unroll
+  for (int p = 0; p < TT / 16; ++p) {
+    const int rl = rq + 16 * p;
+    const int64_t r = r0 + rl, c = c0 + 4 * cq;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < rows && c < cols) x = *reinterpret_cast<const float4*>(src + r * lds + c);
+    t[rl][4 * cq] = x.x;
+    t[rl][4 * cq + 1] = x.y;
+    t[rl][4 * cq + 2] = x.z;
+    t[rl][4 * cq + 3] = x.w;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int p = 0; p < TT / 16; ++p) {
+    const int cl = rq + 16 * p;            // destination row = source column c0 + cl
+    const int64_t c = c0 + cl, r = r0 + 4 * cq;
+    if (c < cols && r < rows) {
+      const float4 x = make_float4(t[4 * cq][cl], t[4 * cq + 1][cl], t[4 * cq + 2][cl], t[4 * cq + 3][cl]);
+      float4 h, l;
+      split4(x, h, l);
+      *reinterpret_cast<float4*>(hi + c * ldd + r) = h;
+      *reinterpret_cast<float4*>(lo + c * ldd + r) = l;
+    }
+  }
+}
+
 void set_attr_once(int device) {
   static bool done[64] = {false};
   if (!done[device & 63]) {
@@ -605,6 +675,23 @@ void set_attr_once(int device) {
 void split_tf32(const Ctx& c, const float* src, int64_t rows, int64_t cols, int64_t lds, float* hi, float* lo,
                 int64_t ldd, bool transpose) {
   if (rows <= 0 || cols <= 0) return;
+  const bool vec = aligned16(src) && aligned16(hi) && aligned16(lo) && lds % 4 == 0 && ldd % 4 == 0 &&
+                   cols % 4 == 0 && (!transpose || rows % 4 == 0);
+  if (vec && transpose && (rows + TT - 1) / TT <= 65535) {
+    dim3 grid(static_cast<unsigned>((cols + TT - 1) / TT), static_cast<unsigned>((rows + TT - 1) / TT));
+    split_tf32_t64_kernel<<<grid, 256, 0, c.stream>>>(src, rows, cols, lds, hi, lo, ldd);
+    check_launch("split_tf32_t64_kernel");
+    return;
+  }
+  if (vec && !transpose) {
+    const int64_t total = rows * (cols / 4);
+    const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(c.sm_count) * 8));
+    split_tf32_v4_kernel<<<grid, 256, 0, c.stream>>>(reinterpret_cast<const float4*>(src), rows, cols / 4, lds / 4,
+                                                     reinterpret_cast<float4*>(hi), reinterpret_cast<float4*>(lo),
+                                                     ldd / 4);
+    check_launch("split_tf32_v4_kernel");
+    return;
+  }
   if (transpose) {
     if ((rows + 31) / 32 > 65535) fail(OC_ERR_INVALID_ARG, "split_tf32: too many rows");
     dim3 grid(static_cast<unsigned>((cols + 31) / 32), static_cast<unsigned>((rows + 31) / 32));

@@ -118,8 +118,6 @@ int finish(const Ctx& c) {
   return st;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 template <class F>
 int guarded(F&& f) {
   try {

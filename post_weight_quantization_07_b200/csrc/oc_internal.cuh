@@ -84,6 +84,8 @@ class PhaseScope {
   bool active_ = false;
 };
 
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 // TMA descriptor for a row-major 2-D array [rows x cols] of `elem_bytes`
 // elements with leading dimension `ld` (elements), box [box_rows x box_cols].
 enum class Swz { None, B128 };
