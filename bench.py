@@ -41,8 +41,8 @@ CPU_SAMPLE_ROWS = 2048
 # DRAM bytes (read + written) per launch of atb_bf16_kernel, the mean of its
 # two launches in one layer, from one ncu capture of dram__bytes_read.sum and
 # dram__bytes_write.sum on this workload at full size (profiles/ has the
-# summary and the command): 33 launches per layer, 19.2 GB in all.
-TRAFFIC_PER_LAUNCH = {"c2_q_proj": 582200250}
+# summary and the command): 33 launches per layer, 20.4 GB in all.
+TRAFFIC_PER_LAUNCH = {"c2_q_proj": 617853192}
 
 
 def load_peaks():
