@@ -548,6 +548,83 @@ def quantize_chain(Ws, x0, alpha: float, damp: float, wbits: int, groupsize: int
     return layers, (x, xh)
 
 
+# ----------------------------------------------------------------------------- LPCD (two-layer submodule)
+#
+# Layer-projected coordinate descent [OneComp-release, section "v1.1.0全新量化方法"
+# (LPCD bullet) and section "量化錯誤傳播 (QEP)"; OneComp-hub, section "3. LPCD：
+# 子模块联合优化"]: related linear layers are quantised together by optimising a
+# relaxed (continuous) objective of the submodule's output, one layer at a time,
+# and projecting each layer's relaxed solution with the layer-wise quantiser.
+# The pages give neither the objective nor the update; the reading taken here is
+# the plainest one for a two-layer linear submodule y = x W1^T W2^T (V/O without
+# the attention mixing, or any two linear layers in sequence):
+#   objective  E(Q1, Q2) = || x W1^T W2^T - xh Q1^T Q2^T ||_F^2
+#   start      the layer-wise method: QEP (alpha) + GPTQ of W1 on (x, xh), then of
+#              W2 on (z, zh) with z = x W1^T, zh = xh Q1^T (bf16 forward products)
+#   each round layer-1 step: with Q2 fixed, the relaxed minimiser of E over Q1
+#              (ridge-regularised on both sides) is
+#                 W1* = (Q2^T Q2 + mu I)^-1 Q2^T W2 . W1 (x^T xh + lam I)(xh^T xh + lam I)^-1
+#              and the second factor is QEP's correction with alpha = 1; GPTQ of
+#              W1* with H1 = 2 xh^T xh projects it.
+#              layer-2 step: with Q1 fixed, the relaxed minimiser over Q2 is QEP's
+#              correction with alpha = 1 on (z, zh); GPTQ with H2 = 2 zh^T zh
+#              projects it.
+#   lam = damp mean(diag(xh^T xh)) as in QEP; mu = damp mean(diag(Q2^T Q2)).
+
+def lpcd_left_project(B, W2, V, damp: float):
+    """(B^T B + mu I)^-1 B^T W2 V with mu = damp * mean(diag(B^T B)): the left
+    factor of LPCD's relaxed layer-1 step (B = the quantised second layer,
+    W2 = its full-precision weights, V = QEP-corrected first layer with
+    alpha = 1).  It is the ridge-regression minimiser of
+    ||B W - W2 V||_F^2 + mu ||W||_F^2 over W (d x n)."""
+    B, W2, V = _f64(B), _f64(W2), _f64(V)
+    M = B.T @ B
+    mu = damp * float(np.mean(np.diag(M)))
+    M = M + mu * np.eye(M.shape[0])
+    return sla.cho_solve(sla.cho_factor(M), B.T @ (W2 @ V))
+
+
+def submodule_error(W1, W2, Q1, Q2, x, xh):
+    """E = ||x W1^T W2^T - xh Q1^T Q2^T||_F^2 and the same for the reference
+    output alone (float64, no rounding)."""
+    y = (_f64(x) @ _f64(W1).T) @ _f64(W2).T
+    yh = (_f64(xh) @ _f64(Q1).T) @ _f64(Q2).T
+    return float(np.sum((y - yh) ** 2)), float(np.sum(y ** 2))
+
+
+def lpcd_pair(W1, W2, x, xh, alpha: float, damp: float, wbits: int, groupsize: int, act_order: bool,
+              rounds: int = 1):
+    """Quantise the two-layer submodule (W1: d x n, W2: m x d) by the reading
+    above: the layer-wise QEP start, then `rounds` rounds of the layer-1 and
+    layer-2 projected steps.  Forward products use bf16 weights and activations
+    and round the product to bf16, as ``quantize_chain`` does.  Returns a dict
+    with the final quantised layers (q1, q2: gptq_quantize outputs), the
+    relaxed layer-1 solutions of each round (W1_star) with the quantised second
+    layer each was solved against (Q2_used), and the submodule error after the
+    start and after every round (errors, ref)."""
+    W1, W2 = _f64(W1), _f64(W2)
+    x, xh = _bf16(x), _bf16(xh)
+    H1 = hessian(xh)
+    q1 = gptq_quantize(qep_correct(W1, x, xh, alpha, damp, H=H1), H1, wbits, groupsize, damp, act_order)
+    z = _bf16(x @ _bf16(W1).T)
+    zh = _bf16(xh @ _bf16(q1["deq"]).T)
+    H2 = hessian(zh)
+    q2 = gptq_quantize(qep_correct(W2, z, zh, alpha, damp, H=H2), H2, wbits, groupsize, damp, act_order)
+    e, ref = submodule_error(W1, W2, q1["deq"], q2["deq"], x, xh)
+    errors, stars, q2_used = [e], [], []
+    V1 = qep_correct(W1, x, xh, 1.0, damp, H=H1)
+    for _ in range(rounds):
+        W1s = lpcd_left_project(q2["deq"], W2, V1, damp)
+        stars.append(W1s)
+        q2_used.append(q2["deq"])
+        q1 = gptq_quantize(W1s, H1, wbits, groupsize, damp, act_order)
+        zh = _bf16(xh @ _bf16(q1["deq"]).T)
+        H2 = hessian(zh)
+        q2 = gptq_quantize(qep_correct(W2, z, zh, 1.0, damp, H=H2), H2, wbits, groupsize, damp, act_order)
+        errors.append(submodule_error(W1, W2, q1["deq"], q2["deq"], x, xh)[0])
+    return {"q1": q1, "q2": q2, "W1_star": stars, "Q2_used": q2_used, "V1": V1, "errors": errors, "ref": ref}
+
+
 # ----------------------------------------------------------------------------- Hadamard rotation
 
 def hadamard(b: int):
