@@ -711,6 +711,72 @@ def run_block(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_lpcd(args, rank, world, local_rank):
+    """LPCD of one Llama-2-7B-shaped V/O pair treated as the linear submodule
+    y = x W_v^T W_o^T (4096x4096 each, 4-bit g128, QEP alpha 0.5 start, damp
+    0.01): the layer-wise start plus --lpcd-rounds rounds of the projected
+    coordinate steps, all inside the timed step.  X, Xhat follow v_proj's
+    recipe; W_v, W_o are seeded N(0, 0.02^2) rounded to bf16.  The submodule's
+    output error before and after the rounds comes from one more, untimed run."""
+    import torch
+
+    import post_weight_quantization_07_b200 as oc
+    from synthetic import llama7b_layers, make_layer_device
+
+    torch.cuda.set_device(local_rank)
+    n_tok = args.n_tok or 131072
+    specs = llama7b_layers(n_tok)
+    sv, so = specs[2], specs[3]
+    L = make_layer_device(sv.with_(seed=sv.seed + 1000 * rank), "cuda")
+    gen = torch.Generator(device="cuda").manual_seed(so.seed + 1000 * rank)
+    Wo = (torch.randn(so.d_out, so.d_in, generator=gen, device="cuda") * so.w_std).to(torch.bfloat16).float()
+    Wv, X, Xh = L["W"], L["X"], L["Xhat"]
+    R = args.lpcd_rounds
+    stream = torch.cuda.current_stream()
+    oc.oc_set_sync(False)
+
+    def step(track=False):
+        return oc.lpcd_pair(Wv, Wo, X, Xh, sv.alpha, sv.damp, sv.wbits, sv.groupsize, sv.act_order, rounds=R,
+                            stream=stream, track_error=track)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    launches0 = oc.oc_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(local_rank)
+    bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+    with ClockSampler(gpu_index_for(local_rank), bus) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    launches = oc.oc_launch_count() - launches0
+    st = oc.oc_stream_status(stream)
+    if st != oc.OC_OK:
+        raise RuntimeError(f"LPCD steps failed: {oc.oc_status_string(st)}")
+    ms = e0.elapsed_time(e1) / args.steps
+    r = step(track=True)
+    rel = [e / r["ref"] for e in r["errors"]]
+    line = {
+        "metric": "LPCD two-layer submodules quantized/sec (Llama-7B V/O shapes, 4-bit g128)",
+        "value": round(world / (ms / 1e3), 4), "unit": "submodules/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16+f32",
+        "data": "synthetic",
+        "config": {"workload": (f"lpcd_vo: Llama-2-7B v_proj and o_proj (4096x4096 each) as the linear "
+                                f"submodule y = x W_v^T W_o^T, {n_tok} calibration tokens (v_proj recipe), "
+                                f"4-bit g128, QEP alpha 0.5 start, damp 0.01, {R} LPCD round(s)"),
+                   "rounds": R, "l2": "inputs larger than L2, no flush needed"},
+        "submodule_rel_error": {"layer_wise_start": round(rel[0], 6),
+                                "after_rounds": [round(x, 6) for x in rel[1:]]},
+        "gpu_launches": int(launches), "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
@@ -758,6 +824,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rotate", type=int, default=0, metavar="B",
                     help="rotate W, X, Xhat by a block-B Hadamard matrix every step before quantising")
+    ap.add_argument("--lpcd-rounds", type=int, default=1,
+                    help="LPCD rounds after the layer-wise start (--workload lpcd_vo)")
     ap.add_argument("--shard-layer", action="store_true",
                     help="one layer split over the ranks (tokens and rows) instead of one layer per rank")
     args = ap.parse_args()
@@ -770,6 +838,8 @@ def main():
         run_reference(args, rank, world)
     elif args.workload == "c4_block":
         run_block(args, rank, world, local_rank)
+    elif args.workload == "lpcd_vo":
+        run_lpcd(args, rank, world, local_rank)
     elif args.shard_layer:
         run_shard_layer(args, rank, world, local_rank)
     else:

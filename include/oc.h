@@ -245,6 +245,30 @@ int oc_quantize_from_terms(const float* W, int64_t m, int64_t n, const float* H,
 int oc_hadamard_rotate(const void* X, int64_t rows, int64_t n, int block, void* Y, int bf16, void* stream);
 
 /*
+ * The relaxed layer-1 step of LPCD (layer-projected coordinate descent) for a
+ * two-layer linear submodule y = x W1^T W2^T (OneComp release summary, LPCD
+ * bullet of section "v1.1.0全新量化方法" and section "量化錯誤傳播 (QEP)"; One
+ * Compression hub page, section "3. LPCD：子模块联合优化": related layers are
+ * optimised together on a relaxed objective and each layer's solution is
+ * projected with the layer-wise quantiser).  With the second layer held at
+ * its quantised value B, the minimiser over the first layer of
+ * ||x W1^T W2^T - xh W^T B^T||^2 (ridge-regularised on both sides) is
+ *   W_out = (B^T B + mu I)^-1 B^T W2 V,   mu = damp * mean(diag(B^T B)),
+ * where V is W1 corrected by QEP with alpha = 1 (oc_qep_correct); GPTQ of
+ * W_out with the first layer's Hessian is the projection.
+ *   B, W2   fp32 [m x d] row-major (quantised and full-precision second layer).
+ *   V       fp32 [d x n] row-major.   W_out fp32 [d x n]; may alias V.
+ *   d       a positive multiple of 64, at most 49152; m, n positive multiples of 4.
+ * Arithmetic: 3xTF32 products on the tensor cores and the library's
+ * inverse-Cholesky factorisation of B^T B + mu I.
+ * Errors: OC_ERR_INVALID_ARG for null or unaligned pointers, bad sizes or a
+ * negative damp; OC_ERR_NOT_SPD when B^T B + mu I is not positive definite
+ * (a zero damp with B of rank below d).
+ */
+int oc_lpcd_left_project(const float* B, const float* W2, int64_t m, int64_t d, const float* V, int64_t n,
+                         float damp, float* W_out, void* stream);
+
+/*
  * Dequantise packed GPTQ output: out[i][j] = scales[i][g] * (q[i][j] - zeros[i][g]),
  * g = j / groupsize, q read from row i's LSB-first bitstream of wbits-bit codes
  * (the layout oc_gptq_quantize writes).  This is the weight the quantised

@@ -44,6 +44,10 @@ Readings taken where the sources leave a step open:
     groups stay contiguous in original order.
   * Packing: per row an LSB-first bitstream of b-bit codes along d_in in original
     column order, stored as uint32 words (b = 3 runs across word boundaries).
+  * LPCD (layer-projected coordinate descent): the pages give no formula; the
+    reading for a two-layer linear submodule is stated above ``lpcd_left_project``.
+    Its functions are pinned to that reading's own mathematics (brute-force least
+    squares); parity against the pages' LPCD itself is unpinned.
 """
 from __future__ import annotations
 

@@ -19,7 +19,8 @@ __all__ = ["OC_OK", "OC_ERR_INVALID_ARG", "OC_ERR_UNSUPPORTED", "OC_ERR_NOT_SPD"
            "LIB_PATH", "HEADER_PATH", "lib", "declared_symbols", "oc_hessian_accumulate",
            "oc_qep_correct", "oc_gptq_quantize", "oc_set_sync", "oc_stream_status",
            "oc_workspace_release", "oc_status_string", "oc_last_error", "oc_version",
-           "oc_profile_enable", "oc_profile_read", "oc_launch_count", "oc_quantize_layer"]
+           "oc_profile_enable", "oc_profile_read", "oc_launch_count", "oc_quantize_layer",
+           "oc_lpcd_left_project", "lpcd_pair"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liboc.so")
@@ -90,6 +91,8 @@ def _load():
     L.oc_quantize_from_terms.restype = i32
     L.oc_hadamard_rotate.argtypes = [vp, i64, i64, i32, vp, i32, vp]
     L.oc_hadamard_rotate.restype = i32
+    L.oc_lpcd_left_project.argtypes = [vp, vp, i64, i64, vp, i64, f32, vp, vp]
+    L.oc_lpcd_left_project.restype = i32
     return L
 
 
@@ -413,6 +416,84 @@ def oc_quantize_from_terms(W, H, D, alpha, damp, wbits, groupsize, act_order, W_
         pp, _stream_handle(stream))
     _check(st, "oc_quantize_from_terms")
     return W_out, codes, scales, zeros, perm_out
+
+
+def oc_lpcd_left_project(B, W2, V, damp, W_out=None, stream=None):
+    """(B^T B + mu I)^-1 B^T W2 V, mu = damp * mean(diag(B^T B)): LPCD's relaxed
+    first-layer step (B, W2 fp32 [m x d]; V fp32 [d x n]; W_out may be V)."""
+    import torch
+    m, d = B.shape
+    d2, n = V.shape
+    if W2.shape != (m, d) or d2 != d:
+        raise ValueError("B and W2 must be [m x d] and V [d x n]")
+    if W_out is None:
+        W_out = torch.empty(d, n, dtype=torch.float32, device=V.device)
+    st = _lib().oc_lpcd_left_project(_dev_ptr(B, torch.float32, "B", (m, d)), _dev_ptr(W2, torch.float32, "W2", (m, d)),
+                                     m, d, _dev_ptr(V, torch.float32, "V", (d, n)), n, float(damp),
+                                     _dev_ptr(W_out, torch.float32, "W_out", (d, n)), _stream_handle(stream))
+    _check(st, "oc_lpcd_left_project")
+    return W_out
+
+
+def lpcd_pair(W1, W2, X, Xhat, alpha, damp, wbits, groupsize, act_order, rounds=1, stream=None,
+              track_error=True):
+    """Quantise a two-layer linear submodule y = x W1^T W2^T by layer-projected
+    coordinate descent (OneComp release summary, LPCD bullet of section
+    "v1.1.0全新量化方法"; hub page section "3. LPCD：子模块联合优化").
+
+    Start: the layer-wise method, oc_quantize_layer of W1 on (X, Xhat) and of
+    W2 on (Z, Zh) with Z = X W1^T and Zh = Xhat Q1^T.  Each round: the relaxed
+    first-layer optimum against the current quantised second layer,
+    oc_lpcd_left_project(Q2, W2, V1) with V1 = oc_qep_correct(W1, alpha = 1),
+    projected by oc_gptq_quantize with the first layer's Hessian; then the
+    second layer again by oc_quantize_layer with alpha = 1 on (Z, Zh).  Forward
+    products are bf16 GEMMs (cuBLAS through torch), as in quantize_chain.
+    W1 fp32 [d x n], W2 fp32 [m x d]; X, Xhat bf16 [N x n].  Returns a dict
+    with the final layers' (codes, scales, zeros, perm) as q1 and q2, their
+    dequantised weights Q1, Q2, the relaxed first-layer weights of each round
+    (W1_star) with the quantised second layer each was solved against
+    (Q2_used), the first layer's Hessian H1 and QEP weights V1 and, with track_error, the submodule's squared output error
+    after the start and each round (errors) and the reference's squared norm.
+    """
+    import torch
+    d, n = W1.shape
+    m = W2.shape[0]
+    X = X.to(torch.bfloat16).contiguous()
+    Xhat = Xhat.to(torch.bfloat16).contiguous()
+    H1, _, c1, s1, z1, p1 = oc_quantize_layer(W1, X, Xhat, alpha, damp, wbits, groupsize, act_order, stream=stream)
+    Q1 = oc_dequantize(c1, s1, z1, n, wbits, groupsize, stream=stream)
+    Z = (X @ W1.to(torch.bfloat16).t()).contiguous()
+
+    def second(Q1, a):
+        Zh = (Xhat @ Q1.to(torch.bfloat16).t()).contiguous()
+        _, _, c2, s2, z2, p2 = oc_quantize_layer(W2, Z, Zh, a, damp, wbits, groupsize, act_order, stream=stream)
+        return (c2, s2, z2, p2), oc_dequantize(c2, s2, z2, d, wbits, groupsize, stream=stream)
+
+    def error(Q1, Q2):
+        y = (X.float() @ W1.t()) @ W2.t()
+        yh = (Xhat.float() @ Q1.t()) @ Q2.t()
+        return float(((y - yh).double() ** 2).sum()), float((y.double() ** 2).sum())
+
+    q2, Q2 = second(Q1, alpha)
+    q1 = (c1, s1, z1, p1)
+    out = {"W1_star": [], "Q2_used": [], "errors": []}
+    if track_error:
+        e, out["ref"] = error(Q1, Q2)
+        out["errors"].append(e)
+    V1 = oc_qep_correct(W1, X, Xhat, 1.0, damp, H_opt=H1, stream=stream)
+    for _ in range(rounds):
+        W1s = oc_lpcd_left_project(Q2, W2, V1, damp, stream=stream)
+        out["W1_star"].append(W1s)
+        out["Q2_used"].append(Q2)
+        perm = torch.empty(n, dtype=torch.int32, device=W1.device)
+        c1, s1, z1, _ = oc_gptq_quantize(W1s, H1, wbits, groupsize, damp, act_order, perm_out=perm, stream=stream)
+        q1 = (c1, s1, z1, perm)
+        Q1 = oc_dequantize(c1, s1, z1, n, wbits, groupsize, stream=stream)
+        q2, Q2 = second(Q1, 1.0)
+        if track_error:
+            out["errors"].append(error(Q1, Q2)[0])
+    out.update(q1=q1, q2=q2, Q1=Q1, Q2=Q2, H1=H1, V1=V1)
+    return out
 
 
 def oc_hadamard_rotate(X, block, out=None, stream=None):

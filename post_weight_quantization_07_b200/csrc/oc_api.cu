@@ -749,6 +749,78 @@ int oc_hadamard_rotate(const void* X, int64_t rows, int64_t n, int block, void* 
   });
 }
 
+int oc_lpcd_left_project(const float* B, const float* W2, int64_t m, int64_t d, const float* V, int64_t n,
+                         float damp, float* W_out, void* stream) {
+  return guarded([&]() -> int {
+    if (!B || !W2 || !V || !W_out) fail(OC_ERR_INVALID_ARG, "B, W2, V, W_out must be non-null");
+    if (d < 64 || d % 64) fail(OC_ERR_INVALID_ARG, "d must be a positive multiple of 64");
+    if (d > 49152) fail(OC_ERR_INVALID_ARG, "d above 49152 is not supported");
+    if (m < 4 || m % 4 || n < 4 || n % 4) fail(OC_ERR_INVALID_ARG, "m and n must be positive multiples of 4");
+    if (m > (int64_t(1) << 30) || n > (int64_t(1) << 30)) fail(OC_ERR_INVALID_ARG, "m or n too large");
+    if (!(damp >= 0.f) || damp > 3.4e38f) fail(OC_ERR_INVALID_ARG, "damp must be finite and >= 0");
+    if (!aligned16(B) || !aligned16(W2) || !aligned16(V) || !aligned16(W_out))
+      fail(OC_ERR_INVALID_ARG, "B, W2, V, W_out must be 16-byte aligned");
+    Ctx c = make_ctx(stream);
+    const size_t dd = static_cast<size_t>(d) * d, dm = static_cast<size_t>(d) * m, dn = static_cast<size_t>(d) * n;
+    Carve sizing{nullptr};
+    sizing.take<float>(dm);                       // B^T hi
+    sizing.take<float>(dm);                       // B^T lo
+    sizing.take<float>(dm);                       // W2^T hi
+    sizing.take<float>(dm);                       // W2^T lo
+    sizing.take<float>(dd);                       // B^T B -> (U^T) hi
+    sizing.take<float>(dd);                       // B^T W2 -> (U^T) lo
+    sizing.take<float>(dd);                       // P hi -> U hi
+    sizing.take<float>(dd);                       // P lo -> U lo
+    sizing.take<float>(dn);                       // V^T hi -> T^T hi -> S^T hi
+    sizing.take<float>(dn);                       // V^T lo -> T^T lo -> S^T lo
+    sizing.take<float>(dn);                       // T -> S
+    sizing.take<float>(dd);                       // factor input -> U
+    sizing.take<float>(dd);                       // inverse factor
+    sizing.take<float>(dd + 4096);                // recursion scratch
+    sizing.take<float>(factor_split_floats(d));   // split copies inside the factorisation
+    sizing.take<DiagStats>(1);
+    Carve cv{workspace(c, sizing.off + 256)};
+    float* Bth = cv.take<float>(dm);
+    float* Btl = cv.take<float>(dm);
+    float* Wth = cv.take<float>(dm);
+    float* Wtl = cv.take<float>(dm);
+    float* Mm = cv.take<float>(dd);
+    float* P = cv.take<float>(dd);
+    float* Ph = cv.take<float>(dd);
+    float* Pl = cv.take<float>(dd);
+    float* Qh = cv.take<float>(dn);
+    float* Ql = cv.take<float>(dn);
+    float* T = cv.take<float>(dn);
+    float* F = cv.take<float>(dd);
+    float* Fx = cv.take<float>(dd);
+    float* Fs = cv.take<float>(dd + 4096);
+    float* fsplit = cv.take<float>(factor_split_floats(d));
+    DiagStats* stats = cv.take<DiagStats>(1);
+    PhaseScope ps(c, kPhLpcdLeft);
+    // M = B^T B and P = B^T W2 (d x d, contraction over the m rows)
+    split_tf32(c, B, m, d, d, Bth, Btl, m, true);
+    split_tf32(c, W2, m, d, d, Wth, Wtl, m, true);
+    gemm_tf32x3(c, d, d, m, 1.f, Bth, Btl, m, Bth, Btl, m, false, Mm, d, kANone);
+    gemm_tf32x3(c, d, d, m, 1.f, Bth, Btl, m, Wth, Wtl, m, false, P, d, kANone);
+    // (M + mu I)^-1 = U^T U, mu = damp mean(diag M)
+    launch_diag_stats(c, Mm, d, damp, 1.0f, false, stats, nullptr);
+    launch_build_reversed(c, Mm, d, nullptr, stats, 1.0f, false, F);
+    factor_inverse_upper(c, F, Fx, Fs, F, d, true, fsplit);
+    // T = P V
+    split_tf32(c, P, d, d, d, Ph, Pl, d);
+    split_tf32(c, V, d, n, n, Qh, Ql, d, true);
+    gemm_tf32x3(c, d, n, d, 1.f, Ph, Pl, d, Qh, Ql, d, false, T, n, kANone);
+    // S = U T (U upper), then W_out = U^T S (U^T lower)
+    split_tf32(c, F, d, d, d, Ph, Pl, d);
+    split_tf32(c, F, d, d, d, Mm, P, d, true);
+    split_tf32(c, T, d, n, n, Qh, Ql, d, true);
+    gemm_tf32x3(c, d, n, d, 1.f, Ph, Pl, d, Qh, Ql, d, false, T, n, kAUpper);
+    split_tf32(c, T, d, n, n, Qh, Ql, d, true);
+    gemm_tf32x3(c, d, n, d, 1.f, Mm, P, d, Qh, Ql, d, false, W_out, n, kALower);
+    return finish(c);
+  });
+}
+
 int oc_dequantize(const uint32_t* codes, const float* scales, const float* zeros, int64_t m, int64_t n, int wbits,
                   int groupsize, void* out, int out_bf16, void* stream) {
   return guarded([&]() -> int {

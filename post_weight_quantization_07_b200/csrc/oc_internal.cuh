@@ -57,6 +57,7 @@ enum Phase : int {
   kPhHessianFix,    // clearing H, mirroring its upper triangle
   kPhQepCrossFix,   // clearing d, subtracting Xhat^T Xhat
   kPhRotate,        // Hadamard rotation
+  kPhLpcdLeft,      // LPCD's relaxed layer-1 step (products, factorisation, solve)
   kNumPhases
 };
 
