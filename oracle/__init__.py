@@ -506,6 +506,15 @@ def dequantize(packed, scales, zeros, wbits: int, groupsize: int, n: int):
     return s * (codes - z)
 
 
+def dequant_gemv(packed, scales, zeros, wbits: int, groupsize: int, n: int, x):
+    """y = x Q^T with Q = dequantize(packed, scales, zeros): the quantised
+    layer applied to a few bf16 activation rows x [batch x n] (the served
+    model's linear layer, One Compression hub page section "4. vLLM 插件：
+    量化模型直接推理": quantised models run inference from their GPTQ codes).
+    Float64; returns [batch x m]."""
+    return _f64(x) @ dequantize(packed, scales, zeros, wbits, groupsize, n).T
+
+
 def _bf16(a):
     """Round to the nearest bf16 value (ties to even), as float64."""
     a32 = np.ascontiguousarray(a, dtype=np.float32)

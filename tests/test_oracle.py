@@ -458,3 +458,23 @@ def test_hadamard_rotation_preserves_layer_output_and_is_an_involution():
         assert np.allclose(oracle.hadamard_rotate(Xr, b), X, rtol=0, atol=1e-12)
         # blocks act independently: the first block of a row only mixes its own b features
         assert np.allclose(Xr[:, :b], X[:, :b] @ (oracle.hadamard(b) / np.sqrt(b)), rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- dequantising GEMV
+
+def test_dequant_gemv_by_explicit_sums():
+    # y[b][i] = sum_j x[b][j] * scale[i][j // G] * (q[i][j] - zero[i][j // G]), summed by loops
+    rng = np.random.default_rng(77)
+    for wbits, G, m, n in [(4, 8, 3, 32), (3, 32, 2, 64), (2, 16, 4, 64)]:
+        codes = rng.integers(0, 2 ** wbits, size=(m, n))
+        scales = rng.uniform(0.5, 2.0, size=(m, n // G))
+        zeros = rng.integers(0, 2 ** wbits, size=(m, n // G)).astype(np.float64)
+        x = rng.standard_normal((3, n))
+        packed = oracle.pack_codes(codes, wbits)
+        y = oracle.dequant_gemv(packed, scales, zeros, wbits, G, n, x)
+        ref = np.zeros((3, m))
+        for b in range(3):
+            for i in range(m):
+                for j in range(n):
+                    ref[b, i] += x[b, j] * scales[i, j // G] * (codes[i, j] - zeros[i, j // G])
+        assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
