@@ -777,6 +777,101 @@ def run_lpcd(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_gemv(args, rank, world, local_rank):
+    """The quantised layers of one Llama-2-7B-shaped block applied at decode
+    time straight from packed codes (oc_dequant_gemv): q/k/v/o 4096x4096 at
+    4 bits, gate/up 4096->11008 and down 11008->4096 at 3 bits, g128, batch
+    --gemv-batch tokens.  Codes, scales and zeros are seeded random values of
+    the quantiser's layout (the GEMV's cost does not depend on them).  The
+    95 MB of codes and grids fit in L2, so every step is timed alone after a
+    write of a buffer larger than L2."""
+    import torch
+
+    import post_weight_quantization_07_b200 as oc
+
+    torch.cuda.set_device(local_rank)
+    nb = args.gemv_batch
+    shapes = [(4096, 4096, 4)] * 4 + [(11008, 4096, 3)] * 2 + [(4096, 11008, 3)]
+    gen = torch.Generator(device="cuda").manual_seed(5150 + rank)
+    layers = []
+    nbytes = 0
+    for m, n, b in shapes:
+        codes = torch.randint(-2 ** 31, 2 ** 31 - 1, (m, n * b // 32), generator=gen, device="cuda",
+                              dtype=torch.int32)
+        scales = torch.rand(m, n // 128, generator=gen, device="cuda") * 0.01 + 1e-3
+        zeros = torch.randint(0, 2 ** b, (m, n // 128), generator=gen, device="cuda").float()
+        x = torch.randn(nb, n, generator=gen, device="cuda").to(torch.bfloat16)
+        y = torch.empty(nb, m, device="cuda")
+        layers.append((codes, scales, zeros, n, b, x, y))
+        nbytes += codes.numel() * 4 + scales.numel() * 4 + zeros.numel() * 4 + x.numel() * 2 + y.numel() * 4
+    oc.oc_set_sync(False)
+
+    def step():
+        # stream=None: the current stream, which is the capture stream below
+        for codes, scales, zeros, n, b, x, y in layers:
+            oc.oc_dequant_gemv(codes, scales, zeros, n, b, 128, x, y=y)
+
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    # A decode loop replays its launches as a CUDA graph; the eager calls'
+    # host overhead (Python, ctypes, argument checks) exceeds these kernels.
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    stream = torch.cuda.current_stream()
+    graph.replay()
+    torch.cuda.synchronize()
+
+    def timed(run):
+        total = 0.0
+        for _ in range(args.steps):
+            flush.fill_(1.0)
+            a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            run()
+            e.record(stream)
+            e.synchronize()
+            total += a.elapsed_time(e)
+        return total / args.steps
+
+    props = torch.cuda.get_device_properties(local_rank)
+    bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+    with ClockSampler(gpu_index_for(local_rank), bus) as clk:
+        ms = timed(graph.replay)
+    launches = 7 * args.steps  # one kernel per layer per replay (the counter sees host calls only)
+    ms_eager = timed(step)
+    st = oc.oc_stream_status(stream)
+    if st != oc.OC_OK:
+        raise RuntimeError(f"GEMV steps failed: {oc.oc_status_string(st)}")
+    del graph
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("hbm_gbs")
+    achieved = nbytes / (ms / 1e3) / 1e9
+    line = {
+        "metric": "dequantising GEMV over packed GPTQ codes: decode steps of one Llama-7B block per second",
+        "value": round(world / (ms / 1e3), 2), "unit": "block-steps/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 (bf16 activations, packed int codes)", "data": "synthetic",
+        "config": {"workload": (f"gemv_block: q/k/v/o 4096x4096 4-bit and gate/up/down 4096<->11008 3-bit, "
+                                f"g128, {nb} token(s) per step"),
+                   "batch": nb, "l2": "flushed before every step (a write of twice L2)"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 3) if peak else None, "traffic": None,
+                     "peak_source": f"{peak_src} copy bandwidth (of {peak_src})", "bytes_per_step": nbytes},
+        "eager_ms_per_step": round(ms_eager, 4), "launch": "CUDA graph replay of the step's 7 calls",
+        "gpu_launches": int(launches), "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
@@ -824,6 +919,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rotate", type=int, default=0, metavar="B",
                     help="rotate W, X, Xhat by a block-B Hadamard matrix every step before quantising")
+    ap.add_argument("--gemv-batch", type=int, default=1,
+                    help="tokens per decode step (--workload gemv_block, 1..8)")
     ap.add_argument("--lpcd-rounds", type=int, default=1,
                     help="LPCD rounds after the layer-wise start (--workload lpcd_vo)")
     ap.add_argument("--shard-layer", action="store_true",
@@ -840,6 +937,8 @@ def main():
         run_block(args, rank, world, local_rank)
     elif args.workload == "lpcd_vo":
         run_lpcd(args, rank, world, local_rank)
+    elif args.workload == "gemv_block":
+        run_gemv(args, rank, world, local_rank)
     elif args.shard_layer:
         run_shard_layer(args, rank, world, local_rank)
     else:

@@ -284,6 +284,23 @@ int oc_dequantize(const uint32_t* codes, const float* scales, const float* zeros
                   int wbits, int groupsize, void* out, int out_bf16, void* stream);
 
 /*
+ * The quantised layer applied to a few activation rows straight from its
+ * packed codes: y[b][i] = sum_j x[b][j] * scales[i][g] * (q[i][j] - zeros[i][g]),
+ * g = j / groupsize (One Compression hub page, section "4. vLLM 插件：量化模型直接
+ * 推理": quantised GPTQ models are served by inference from their codes; at
+ * decode time a layer is a matrix-vector product whose cost is reading them).
+ *   codes   uint32 [m x n*wbits/32], the layout oc_gptq_quantize writes.
+ *   scales, zeros fp32 [m x n/groupsize].
+ *   x       bf16 [batch x n] row-major, batch 1..8.    y fp32 [batch x m].
+ *   n       a positive multiple of 32; groupsize dividing both n and 32, a
+ *           multiple of 32 dividing n, or -1 (= n).
+ * fp32 products and sums; one warp per output row reads the row's codes once.
+ * Errors: OC_ERR_INVALID_ARG for null or unaligned codes/x, bad sizes or groups.
+ */
+int oc_dequant_gemv(const uint32_t* codes, const float* scales, const float* zeros, int64_t m, int64_t n,
+                    int wbits, int groupsize, const void* x, int64_t batch, float* y, void* stream);
+
+/*
  * Several layers that read the same calibration inputs, e.g. the q, k and v
  * projections of one attention block or gate and up of one MLP (the One
  * Compression hub page, section "核心功能拆解", quantises a model layer by

@@ -20,7 +20,7 @@ __all__ = ["OC_OK", "OC_ERR_INVALID_ARG", "OC_ERR_UNSUPPORTED", "OC_ERR_NOT_SPD"
            "oc_qep_correct", "oc_gptq_quantize", "oc_set_sync", "oc_stream_status",
            "oc_workspace_release", "oc_status_string", "oc_last_error", "oc_version",
            "oc_profile_enable", "oc_profile_read", "oc_launch_count", "oc_quantize_layer",
-           "oc_lpcd_left_project", "lpcd_pair"]
+           "oc_lpcd_left_project", "lpcd_pair", "oc_dequant_gemv"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liboc.so")
@@ -93,6 +93,8 @@ def _load():
     L.oc_hadamard_rotate.restype = i32
     L.oc_lpcd_left_project.argtypes = [vp, vp, i64, i64, vp, i64, f32, vp, vp]
     L.oc_lpcd_left_project.restype = i32
+    L.oc_dequant_gemv.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, i64, vp, vp]
+    L.oc_dequant_gemv.restype = i32
     return L
 
 
@@ -433,6 +435,24 @@ def oc_lpcd_left_project(B, W2, V, damp, W_out=None, stream=None):
                                      _dev_ptr(W_out, torch.float32, "W_out", (d, n)), _stream_handle(stream))
     _check(st, "oc_lpcd_left_project")
     return W_out
+
+
+def oc_dequant_gemv(codes, scales, zeros, n, wbits, groupsize, x, y=None, stream=None):
+    """y = x Q^T with Q the dequantised weight of packed codes [m x n*wbits/32];
+    x bf16 [batch x n] (batch 1..8), y fp32 [batch x m]."""
+    import torch
+    m = codes.shape[0]
+    nb = x.shape[0]
+    ng = scales.shape[1]
+    if y is None:
+        y = torch.empty(nb, m, dtype=torch.float32, device=codes.device)
+    st = _lib().oc_dequant_gemv(_dev_ptr(codes, torch.int32, "codes", (m, n * wbits // 32)),
+                                _dev_ptr(scales, torch.float32, "scales", (m, ng)),
+                                _dev_ptr(zeros, torch.float32, "zeros", (m, ng)), m, n, int(wbits),
+                                int(groupsize), _dev_ptr(x, torch.bfloat16, "x", (nb, n)), nb,
+                                _dev_ptr(y, torch.float32, "y", (nb, m)), _stream_handle(stream))
+    _check(st, "oc_dequant_gemv")
+    return y
 
 
 def lpcd_pair(W1, W2, X, Xhat, alpha, damp, wbits, groupsize, act_order, rounds=1, stream=None,

@@ -821,6 +821,27 @@ int oc_lpcd_left_project(const float* B, const float* W2, int64_t m, int64_t d, 
   });
 }
 
+int oc_dequant_gemv(const uint32_t* codes, const float* scales, const float* zeros, int64_t m, int64_t n, int wbits,
+                    int groupsize, const void* x, int64_t batch, float* y, void* stream) {
+  return guarded([&]() -> int {
+    if (!codes || !scales || !zeros || !x || !y) fail(OC_ERR_INVALID_ARG, "codes, scales, zeros, x, y must be non-null");
+    if (m < 1 || n < 32 || n % 32) fail(OC_ERR_INVALID_ARG, "m must be >= 1 and n a positive multiple of 32");
+    if (wbits < 2 || wbits > 4) fail(OC_ERR_INVALID_ARG, "wbits must be 2, 3 or 4");
+    if (batch < 1 || batch > 8) fail(OC_ERR_INVALID_ARG, "batch must be 1..8");
+    const int64_t G = (groupsize == -1) ? n : groupsize;
+    if (G < 1 || n % G) fail(OC_ERR_INVALID_ARG, "groupsize must divide n (or be -1)");
+    if (G < 32 ? (32 % G != 0) : (G % 32 != 0))
+      fail(OC_ERR_INVALID_ARG, "groupsize must divide 32 or be a multiple of 32");
+    if (!aligned16(codes) || !aligned16(x)) fail(OC_ERR_INVALID_ARG, "codes and x must be 16-byte aligned");
+    Ctx c = make_ctx(stream);
+    {
+      PhaseScope ps(c, kPhGemv);
+      launch_dequant_gemv(c, codes, scales, zeros, m, n, wbits, G, x, static_cast<int>(batch), y);
+    }
+    return finish(c);
+  });
+}
+
 int oc_dequantize(const uint32_t* codes, const float* scales, const float* zeros, int64_t m, int64_t n, int wbits,
                   int groupsize, void* out, int out_bf16, void* stream) {
   return guarded([&]() -> int {

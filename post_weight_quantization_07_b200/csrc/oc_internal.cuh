@@ -58,6 +58,7 @@ enum Phase : int {
   kPhQepCrossFix,   // clearing d, subtracting Xhat^T Xhat
   kPhRotate,        // Hadamard rotation
   kPhLpcdLeft,      // LPCD's relaxed layer-1 step (products, factorisation, solve)
+  kPhGemv,          // dequantising GEMV over packed codes
   kNumPhases
 };
 
@@ -194,6 +195,9 @@ void launch_sweep_block(const Ctx& c, float* Wp, int64_t m, int64_t n, const flo
 // Y = X (I (x) H_b) / sqrt(b) along rows of n features, b = 2^log2b <= 4096.
 void launch_hadamard(const Ctx& c, const void* X, void* Y, int64_t rows, int64_t n, int log2b, bool bf16);
 // out[i][j] = scale * (code - zero), fp32 or bf16, original column order.
+// y[b][i] = sum_j x[b][j] Q[i][j] over packed codes (nb <= 8 bf16 rows of x, fp32 y).
+void launch_dequant_gemv(const Ctx& c, const uint32_t* codes, const float* scales, const float* zeros, int64_t m,
+                         int64_t n, int wbits, int64_t G, const void* x, int nb, float* y);
 void launch_dequant(const Ctx& c, const uint32_t* codes, const float* scales, const float* zeros, int64_t m,
                     int64_t n, int wbits, int64_t G, void* out, bool bf16);
 void launch_pack(const Ctx& c, const unsigned char* codes8, int64_t m, int64_t n, int wbits,

@@ -527,3 +527,60 @@ def test_hadamard_rotation_in_place_and_layer_output_invariance():
     torch.cuda.synchronize()
     got = Wr.double() @ X.double().t()
     assert float((got - ref.double()).abs().max()) <= 1e-3 * float(ref.abs().max())
+
+
+# ----------------------------------------------------------------------------- dequantising GEMV
+
+def _gemv_case(m, n, wbits, G, nb, seed):
+    rng = np.random.default_rng(seed)
+    Gs = n if G == -1 else G
+    codes = rng.integers(0, 2 ** wbits, size=(m, n))
+    scales = rng.uniform(0.001, 0.02, size=(m, n // Gs)).astype(np.float32)
+    zeros = rng.integers(0, 2 ** wbits, size=(m, n // Gs)).astype(np.float32)
+    x = oracle._bf16(rng.standard_normal((nb, n)))
+    return oracle.pack_codes(codes, wbits), scales, zeros, x
+
+
+def _gemv_bound(packed, scales, zeros, wbits, G, n, x):
+    # fp32: one rounding of each dequantised weight and of each product, n
+    # additions: |error| <= gamma_{n+2} * sum_j |x_j q_ij|, gamma_k = k u / (1 - k u)
+    Q = oracle.dequantize(packed, scales, zeros, wbits, G, n)
+    u = 2.0 ** -24
+    k = n + 2
+    return (k * u / (1 - k * u)) * (np.abs(x) @ np.abs(Q).T)
+
+
+@pytest.mark.parametrize("m,n,wbits,G,nb", [
+    (37, 320, 4, 32, 1),
+    (64, 4096, 4, 128, 8),
+    (33, 192, 3, 64, 3),
+    (16, 96, 3, -1, 2),
+    (40, 256, 2, 16, 5),     # groups smaller than a 32-column segment
+    (8, 128, 2, 4, 4),
+    (300, 1024, 3, 8, 1),
+])
+def test_dequant_gemv_matches_oracle(m, n, wbits, G, nb):
+    packed, scales, zeros, x = _gemv_case(m, n, wbits, G, nb, seed=m + n + wbits)
+    y = oc.oc_dequant_gemv(dev(packed.view(np.int32), torch.int32), dev(scales), dev(zeros), n, wbits, G,
+                           dev(x, torch.bfloat16)).cpu().numpy()
+    ref = oracle.dequant_gemv(packed, scales, zeros, wbits, G, n, x)
+    assert np.all(np.abs(y - ref) <= _gemv_bound(packed, scales, zeros, wbits, G, n, x))
+
+
+def test_dequant_gemv_on_quantiser_output():
+    L = random_layer_host(96, 512, 1024, seed=4321)
+    H = oracle.hessian(L["Xhat"]).astype(np.float32)
+    codes, scales, zeros, _ = oc.oc_gptq_quantize(dev(L["W"]), dev(H), 3, 128, 0.01, False)
+    x = L["X"][:6]
+    y = oc.oc_dequant_gemv(codes, scales, zeros, 512, 3, 128, bf16_dev(x)).cpu().numpy()
+    p, s, z = codes.cpu().numpy().view(np.uint32), scales.cpu().numpy(), zeros.cpu().numpy()
+    ref = oracle.dequant_gemv(p, s, z, 3, 128, 512, x)
+    assert np.all(np.abs(y - ref) <= _gemv_bound(p, s, z, 3, 128, 512, x))
+
+
+def test_dequant_gemv_rejects_bad_arguments():
+    packed, scales, zeros, x = _gemv_case(8, 96, 4, 32, 9, seed=5)
+    with pytest.raises(oc.OcError) as e:   # batch 9 > 8
+        oc.oc_dequant_gemv(dev(packed.view(np.int32), torch.int32), dev(scales), dev(zeros), 96, 4, 32,
+                           dev(x, torch.bfloat16))
+    assert e.value.status == oc.OC_ERR_INVALID_ARG
