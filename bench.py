@@ -42,7 +42,7 @@ CPU_SAMPLE_ROWS = 2048
 # two launches in one layer, from one ncu capture of dram__bytes_read.sum and
 # dram__bytes_write.sum on this workload at full size (profiles/ has the
 # summary and the command): 33 launches per layer, 20.4 GB in all.
-TRAFFIC_PER_LAUNCH = {"c2_q_proj": 617853192}
+TRAFFIC_PER_LAUNCH = {"q_proj_4096": 617853192}
 
 
 def load_peaks():
@@ -55,10 +55,10 @@ def load_peaks():
 
 
 WORKLOAD_TITLES = {
-    "c1_512": "single 512x512 linear layer",
-    "c2_q_proj": "Llama-2-7B q_proj layer",
-    "c3_down_proj": "Llama-2-7B MLP down_proj layer",
-    "c5_70b_down": "Llama-3-70B-shaped MLP down_proj layer",
+    "layer_512": "single 512x512 linear layer",
+    "q_proj_4096": "Llama-2-7B q_proj layer",
+    "down_proj_11008": "Llama-2-7B MLP down_proj layer",
+    "down_proj_28672": "Llama-3-70B-shaped MLP down_proj layer",
 }
 X_KINDS = {"normal": "N(0,1)", "t": "Student-t({nu:g})", "swiglu": "SiLU(z1)*z2"}
 
@@ -698,7 +698,7 @@ def run_block(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_block, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16+f32",
         "data": "synthetic",
-        "config": {"workload": (f"c4_block: one Llama-2-7B-shaped block (q/k/v/o 4096x4096 4-bit, gate/up "
+        "config": {"workload": (f"block_7b: one Llama-2-7B-shaped block (q/k/v/o 4096x4096 4-bit, gate/up "
                                 f"4096->11008 and down 11008->4096 3-bit, g128, QEP alpha 0.5, damp 0.01), "
                                 f"{n_tok} calibration tokens per input, q/k/v and gate/up sharing their "
                                 f"inputs (one Hessian, cross term and factorisation per group)"),
@@ -878,6 +878,11 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     from synthetic import CONFIGS
+    if args.workload not in CONFIGS:
+        print(json.dumps({"impl": "reference", "unavailable": (
+            f"the float64 oracle arm times single-layer workloads ({', '.join(sorted(CONFIGS))}); "
+            f"{args.workload} has none")}), flush=True)
+        return
     spec = CONFIGS[args.workload]
     if args.n_tok:
         spec = spec.with_(n_tok=args.n_tok)
@@ -912,7 +917,7 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="c2_q_proj")
+    ap.add_argument("--workload", default="q_proj_4096")
     ap.add_argument("--n-tok", type=int, default=None,
                     help="calibration tokens per layer (default: the workload's own)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -933,7 +938,7 @@ def main():
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args, rank, world)
-    elif args.workload == "c4_block":
+    elif args.workload == "block_7b":
         run_block(args, rank, world, local_rank)
     elif args.workload == "lpcd_vo":
         run_lpcd(args, rank, world, local_rank)

@@ -12,17 +12,17 @@ Every workload is one linear layer ``y = W x`` with ``W`` of shape
 quantised layer sees: the full-precision input plus a small channel-wise
 perturbation standing in for the quantisation error of earlier layers.
 
-* ``c1_512``        512 x 512, W fp32 ~ N(0, 1/512); X: 2048 tokens, N(0,1) with 4
-                     random channels x10; X-hat = X + N(0, 0.05^2); 4-bit, g128.
-* ``c2_q_proj``     Llama-2-7B q_proj, 4096 x 4096, W bf16 ~ N(0, 0.02^2); X: 262144
-                     tokens of Student-t(4) with 1% of channels x20; 4-bit g128.
-* ``c3_down_proj``  Llama-2-7B down_proj, d_in 11008, d_out 4096; X: 262144 tokens of
-                     SiLU(z1)*z2 with 0.5% of channels x50; 3-bit g128, act_order.
-* ``c4_llama7b``    224 layers of a 32-block Llama-2-7B-shaped model, 131072 tokens
-                     per layer, Student-t(4) with 1% of channels x20; attention 4-bit,
-                     MLP 3-bit, g128.
-* ``c5_70b_down``   Llama-3-70B down_proj, d_in 28672, d_out 8192; X: 65536 tokens of
-                     Student-t(3) with 1% of channels x30; 2-bit g64, act_order.
+* ``layer_512``        512 x 512, W fp32 ~ N(0, 1/512); X: 2048 tokens, N(0,1) with 4
+                       random channels x10; X-hat = X + N(0, 0.05^2); 4-bit, g128.
+* ``q_proj_4096``      Llama-2-7B q_proj, 4096 x 4096, W bf16 ~ N(0, 0.02^2); X: 262144
+                       tokens of Student-t(4) with 1% of channels x20; 4-bit g128.
+* ``down_proj_11008``  Llama-2-7B down_proj, d_in 11008, d_out 4096; X: 262144 tokens of
+                       SiLU(z1)*z2 with 0.5% of channels x50; 3-bit g128, act_order.
+* ``llama7b_layers``   224 layers of a 32-block Llama-2-7B-shaped model, 131072 tokens
+                       per layer, Student-t(4) with 1% of channels x20; attention 4-bit,
+                       MLP 3-bit, g128.
+* ``down_proj_28672``  Llama-3-70B down_proj, d_in 28672, d_out 8192; X: 65536 tokens of
+                       Student-t(3) with 1% of channels x30; 2-bit g64, act_order.
 
 Readings where the workload description leaves a knob open (each listed in the
 design notes): outlier channel count is ``max(1, floor(frac * d_in))``, chosen
@@ -59,7 +59,7 @@ class LayerSpec:
     n_outliers: int = 0     # used when outlier_frac == 0
     outlier_scale: float = 1.0
     noise_abs: float = 0.0  # X-hat = X + N(0, noise_abs^2)          (c1)
-    noise_rel: float = 0.0  # X-hat = X + N(0, (noise_rel*sigma_c)^2)  (c2..c5)
+    noise_rel: float = 0.0  # X-hat = X + N(0, (noise_rel*sigma_c)^2)  (the large workloads)
     wbits: int = 4
     groupsize: int = 128
     act_order: bool = False
@@ -77,19 +77,19 @@ class LayerSpec:
 
 
 CONFIGS = {
-    "c1_512": LayerSpec("c1_512", d_in=512, d_out=512, n_tok=2048,
+    "layer_512": LayerSpec("layer_512", d_in=512, d_out=512, n_tok=2048,
                         w_std=math.sqrt(1.0 / 512), w_bf16=False, x_kind="normal",
                         n_outliers=4, outlier_scale=10.0, noise_abs=0.05,
                         wbits=4, groupsize=128, act_order=False, seed=1),
-    "c2_q_proj": LayerSpec("c2_q_proj", d_in=4096, d_out=4096, n_tok=262144,
+    "q_proj_4096": LayerSpec("q_proj_4096", d_in=4096, d_out=4096, n_tok=262144,
                            w_std=0.02, w_bf16=True, x_kind="t", nu=4.0,
                            outlier_frac=0.01, outlier_scale=20.0, noise_rel=0.02,
                            wbits=4, groupsize=128, act_order=False, seed=2),
-    "c3_down_proj": LayerSpec("c3_down_proj", d_in=11008, d_out=4096, n_tok=262144,
+    "down_proj_11008": LayerSpec("down_proj_11008", d_in=11008, d_out=4096, n_tok=262144,
                               w_std=0.02, w_bf16=True, x_kind="swiglu",
                               outlier_frac=0.005, outlier_scale=50.0, noise_rel=0.02,
                               wbits=3, groupsize=128, act_order=True, seed=3),
-    "c5_70b_down": LayerSpec("c5_70b_down", d_in=28672, d_out=8192, n_tok=65536,
+    "down_proj_28672": LayerSpec("down_proj_28672", d_in=28672, d_out=8192, n_tok=65536,
                              w_std=0.015, w_bf16=True, x_kind="t", nu=3.0,
                              outlier_frac=0.01, outlier_scale=30.0, noise_rel=0.02,
                              wbits=2, groupsize=64, act_order=True, seed=5),
@@ -107,7 +107,7 @@ def llama7b_layers(n_tok: int = 131072):
     for blk in range(32):
         for j, (nm, d_in, d_out, bits) in enumerate(shapes):
             idx = blk * len(shapes) + j
-            out.append(LayerSpec(f"c4_b{blk}_{nm}", d_in=d_in, d_out=d_out, n_tok=n_tok,
+            out.append(LayerSpec(f"l7b_b{blk}_{nm}", d_in=d_in, d_out=d_out, n_tok=n_tok,
                                  w_std=0.02, w_bf16=True, x_kind="t", nu=4.0,
                                  outlier_frac=0.01, outlier_scale=20.0, noise_rel=0.02,
                                  wbits=bits, groupsize=128, act_order=False,

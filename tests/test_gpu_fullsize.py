@@ -25,7 +25,7 @@ oc = pytest.importorskip("post_weight_quantization_07_b200")
 
 pytestmark = pytest.mark.gpu
 
-SPEC = CONFIGS["c2_q_proj"]
+SPEC = CONFIGS["q_proj_4096"]
 CHUNK = 8192
 N_ROWS = 32  # rows replayed by the oracle sweep
 

@@ -25,8 +25,8 @@ pytestmark = pytest.mark.gpu
 CHUNK = 8192
 # (workload, calibration tokens for the oracle comparison, rows replayed, QEP rows)
 CASES = {
-    "c3_down_proj": (16384, 32, None),
-    "c5_70b_down": (8192, 8, 16),
+    "down_proj_11008": (16384, 32, None),
+    "down_proj_28672": (8192, 8, 16),
 }
 
 

@@ -256,7 +256,7 @@ def test_gptq_nonfinite_reports_error():
 # ----------------------------------------------------------------------------- end to end
 
 def test_end_to_end_512_workload():
-    spec = CONFIGS["c1_512"]
+    spec = CONFIGS["layer_512"]
     L = make_layer_host(spec)
     W, X, Xh = L["W"].astype(np.float64), L["X"], L["Xhat"]
     # oracle

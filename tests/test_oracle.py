@@ -358,12 +358,12 @@ def test_teacher_forcing_accepts_own_output_and_flags_planted_error():
 
 
 def test_workload_recipes_shapes():
-    L = make_layer_host(CONFIGS["c1_512"])
+    L = make_layer_host(CONFIGS["layer_512"])
     assert L["W"].shape == (512, 512) and L["X"].shape == (2048, 512)
     assert len(L["outliers"]) == 4
-    assert CONFIGS["c2_q_proj"].outlier_count() == 40
-    assert CONFIGS["c3_down_proj"].outlier_count() == 55
-    assert CONFIGS["c5_70b_down"].outlier_count() == 286
+    assert CONFIGS["q_proj_4096"].outlier_count() == 40
+    assert CONFIGS["down_proj_11008"].outlier_count() == 55
+    assert CONFIGS["down_proj_28672"].outlier_count() == 286
 
 
 def test_qep_precomputed_terms_over_chunks():
