@@ -75,3 +75,36 @@ def test_qep_rejects_bad_arguments():
     assert st == oc.OC_ERR_INVALID_ARG
     st = oc.lib.oc_qep_correct(NULL, 8, 64, FAKE, FAKE, 10, 0.5, 0.01, NULL, FAKE, NULL)
     assert st == oc.OC_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("args,why", [
+    ((NULL, FAKE, 64, 128, FAKE, 32, 0.01, FAKE, NULL), "null B"),
+    ((FAKE, FAKE, 64, 100, FAKE, 32, 0.01, FAKE, NULL), "d not a multiple of 64"),
+    ((FAKE, FAKE, 6, 128, FAKE, 32, 0.01, FAKE, NULL), "m not a multiple of 4"),
+    ((FAKE, FAKE, 64, 128, FAKE, 0, 0.01, FAKE, NULL), "empty n"),
+    ((FAKE, FAKE, 64, 128, FAKE, 32, -1.0, FAKE, NULL), "negative damp"),
+    ((FAKE, FAKE, 64, 128, ctypes.c_void_p((1 << 20) + 4), 32, 0.01, FAKE, NULL), "unaligned V"),
+])
+def test_lpcd_left_project_rejects_bad_arguments(args, why):
+    assert oc.lib.oc_lpcd_left_project(*args) == oc.OC_ERR_INVALID_ARG, why
+    assert oc.oc_last_error() != ""
+
+
+@pytest.mark.parametrize("kw,why", [
+    (dict(codes=NULL), "null codes"),
+    (dict(n=48), "n not a multiple of 32"),
+    (dict(wbits=5), "wbits"),
+    (dict(batch=0), "empty batch"),
+    (dict(batch=9), "batch above 8"),
+    (dict(groupsize=48, n=96), "group of 32 or more that is not a multiple of 32"),
+    (dict(groupsize=12), "group below 32 that does not divide 32"),
+    (dict(groupsize=64, n=96), "group that does not divide n"),
+    (dict(x=ctypes.c_void_p((1 << 20) + 2)), "unaligned x"),
+])
+def test_dequant_gemv_rejects_bad_arguments(kw, why):
+    a = dict(codes=FAKE, scales=FAKE, zeros=FAKE, m=8, n=128, wbits=4, groupsize=32, x=FAKE, batch=1, y=FAKE,
+             stream=NULL)
+    a.update(kw)
+    st = oc.lib.oc_dequant_gemv(a["codes"], a["scales"], a["zeros"], a["m"], a["n"], a["wbits"], a["groupsize"],
+                                a["x"], a["batch"], a["y"], a["stream"])
+    assert st == oc.OC_ERR_INVALID_ARG, why
