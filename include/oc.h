@@ -294,7 +294,8 @@ int oc_dequantize(const uint32_t* codes, const float* scales, const float* zeros
  *   x       bf16 [batch x n] row-major, batch 1..8.    y fp32 [batch x m].
  *   n       a positive multiple of 32; groupsize dividing both n and 32, a
  *           multiple of 32 dividing n, or -1 (= n).
- * fp32 products and sums; one warp per output row reads the row's codes once.
+ * fp32 products and sums; each warp takes four output rows (two with more than
+ * four activation rows) and reads their codes once.
  * Errors: OC_ERR_INVALID_ARG for null or unaligned codes/x, bad sizes or groups.
  */
 int oc_dequant_gemv(const uint32_t* codes, const float* scales, const float* zeros, int64_t m, int64_t n,
