@@ -515,12 +515,27 @@ def dequant_gemv(packed, scales, zeros, wbits: int, groupsize: int, n: int, x):
     return _f64(x) @ dequantize(packed, scales, zeros, wbits, groupsize, n).T
 
 
+_BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127   # largest finite bf16 number
+
+
 def _bf16(a):
-    """Round to the nearest bf16 value (ties to even), as float64."""
-    a32 = np.ascontiguousarray(a, dtype=np.float32)
-    u = a32.view(np.uint32).astype(np.uint64)
-    r = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
-    return r.view(np.float32).astype(np.float64)
+    """Round every value to the nearest bf16 number, ties to even, in one step
+    from float64 (no intermediate float32).  bf16 has 8 significant bits and
+    the float32 exponent range: a normal value x = m 2^e (0.5 <= |m| < 1) is
+    rounded to a multiple of 2^(e-8); below the smallest normal 2^-126 the
+    spacing stays 2^-133 (subnormals).  Results beyond the largest finite bf16
+    become +-inf, as round-to-nearest overflow does; zeros (with their sign),
+    infinities and NaN pass through.  Returns float64."""
+    x = _f64(a)
+    out = np.array(x, dtype=np.float64, copy=True)
+    fin = np.isfinite(x) & (x != 0.0)
+    v = x[fin]
+    _, e = np.frexp(v)
+    q = np.maximum(e - 8, -133)          # exponent of the spacing at v
+    y = np.ldexp(np.rint(np.ldexp(v, -q)), q)   # scaling by 2^-q is exact; rint ties to even
+    y = np.where(np.abs(y) > _BF16_MAX, np.copysign(np.inf, y), y)
+    out[fin] = y
+    return out
 
 
 def _act(y, act: str):

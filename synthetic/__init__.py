@@ -24,8 +24,7 @@ perturbation standing in for the quantisation error of earlier layers.
 * ``down_proj_28672``  Llama-3-70B down_proj, d_in 28672, d_out 8192; X: 65536 tokens of
                        Student-t(3) with 1% of channels x30; 2-bit g64, act_order.
 
-Readings where the workload description leaves a knob open (each listed in the
-design notes): outlier channel count is ``max(1, floor(frac * d_in))``, chosen
+Readings where the workload description leaves a knob open: outlier channel count is ``max(1, floor(frac * d_in))``, chosen
 without replacement; Student-t is the standard t_nu (no rescaling); X-hat for
 the large workloads is ``X + N(0, (0.02 * sigma_c)^2)`` with ``sigma_c`` the
 theoretical standard deviation of channel ``c`` after outlier scaling; X and

@@ -478,3 +478,72 @@ def test_dequant_gemv_by_explicit_sums():
                 for j in range(n):
                     ref[b, i] += x[b, j] * scales[i, j // G] * (codes[i, j] - zeros[i, j // G])
         assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def _bf16_bits(y):
+    b = np.asarray(y, dtype=np.float32).view(np.uint32)
+    assert np.all((b & 0xFFFF) == 0), "result is not a bf16 number"
+    return b >> 16
+
+
+def test_bf16_rounding_hand_worked_bit_patterns():
+    # tests/golden/bf16_rounding.json: ties to even, a tie that a detour
+    # through float32 would break the wrong way, carries into the exponent,
+    # the largest finite value and overflow, subnormals and signed zeros
+    with open(os.path.join(GOLDEN, "bf16_rounding.json")) as f:
+        cases = json.load(f)["cases"]
+    xs = np.array([float(c["x"]) if c["x"].endswith("inf") else float.fromhex(c["x"]) for c in cases])
+    want = np.array([int(c["bits"], 16) for c in cases], dtype=np.uint32)
+    got = _bf16_bits(oracle._bf16(xs))
+    bad = [(c["x"], hex(int(g)), c["bits"]) for c, g, w in zip(cases, got, want) if g != w]
+    assert not bad, bad
+    assert np.isnan(oracle._bf16(np.array([np.nan]))[0])
+
+
+def test_bf16_rounding_fixture_catches_planted_mistakes():
+    # Each plausible slip in a rounding routine fails at least one fixture case.
+    with open(os.path.join(GOLDEN, "bf16_rounding.json")) as f:
+        cases = json.load(f)["cases"]
+    fin = [c for c in cases if not c["x"].endswith("inf")]
+    xs = np.array([float.fromhex(c["x"]) for c in fin])
+    want = np.array([int(c["bits"], 16) for c in fin], dtype=np.uint32)
+
+    def via_float32(a):      # two roundings: float64 -> float32 -> bf16
+        u = np.asarray(a, np.float32).view(np.uint32).astype(np.uint64)
+        return ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32).view(np.float32)
+
+    def ties_away(a):        # ties away from zero instead of to even
+        u = np.asarray(a, np.float32).view(np.uint32).astype(np.uint64)
+        return ((u + 0x8000) & 0xFFFF0000).astype(np.uint32).view(np.float32)
+
+    def truncate(a):         # chopping the low bits
+        u = np.asarray(a, np.float32).view(np.uint32)
+        return (u & np.uint32(0xFFFF0000)).view(np.float32)
+
+    for wrong in (via_float32, ties_away, truncate):
+        got = np.asarray(wrong(xs), np.float32).view(np.uint32) >> 16
+        assert np.any(got != want), wrong.__name__
+
+
+def test_layer_errors_hand_worked():
+    # tests/golden/layer_errors_tiny.json: a 2 x 3 layer on 4 tokens with every
+    # product written out by hand
+    with open(os.path.join(GOLDEN, "layer_errors_tiny.json")) as f:
+        g = json.load(f)
+    W, Q, Wp = (np.array(g[k], dtype=np.float64) for k in ("W", "Q", "W_prime"))
+    X, Xh = np.array(g["X"], dtype=np.float64), np.array(g["Xhat"], dtype=np.float64)
+    e = oracle.layer_errors(W, Q, X, Xh, W_prime=Wp)
+    assert abs(e["e_lit"] ** 2 - g["e_lit_sq"]) <= 1e-12 * g["e_lit_sq"]
+    assert abs(e["e_qep"] ** 2 - g["e_qep_sq"]) <= 1e-12 * g["e_qep_sq"]
+    assert abs(e["e_gptq"] ** 2 - g["e_gptq_sq"]) <= 1e-12 * g["e_gptq_sq"]
+    # the fixture tells the inputs apart: exchanging X and Xhat gives the
+    # hand-worked 'swapped' values, none equal to the right ones
+    s = oracle.layer_errors(W, Q, Xh, X, W_prime=Wp)
+    sw = g["swapped"]
+    assert abs(s["e_lit"] ** 2 - sw["e_lit_sq_with_Xhat"]) <= 1e-12 * 64
+    assert abs(s["e_qep"] ** 2 - sw["e_qep_sq_with_X_and_Xhat_exchanged"]) <= 1e-12 * 64
+    assert abs(s["e_gptq"] ** 2 - sw["e_gptq_sq_with_X"]) <= 1e-12 * 64
+    assert len({g["e_lit_sq"], sw["e_lit_sq_with_Xhat"]}) == 2
+    # a transposed operand cannot be evaluated on these shapes
+    with pytest.raises(ValueError):
+        oracle.layer_errors(W.T, Q.T, X, Xh)
