@@ -345,11 +345,14 @@ int oc_quantize_layer_group(int count, const float* const* W, const int64_t* m, 
  *     needed in oc_last_error().
  *   - The first call on a device looks up the array's device address on that
  *     device (the device must be current); make that first call before any
- *     stream capture begins.
+ *     stream capture begins.  The address is looked up again only if the
+ *     device's context was destroyed and re-created in between.
  *   - Every call on a device shares the one array, which keeps the previous
  *     call's contents (each call clears what must start at zero).  Calls that
- *     overlap on the GPU -- on different streams or from different threads --
- *     race on it and must not be issued.
+ *     overlap on the GPU -- on different streams, or issued from different
+ *     threads without waiting for the previous call's stream -- race on it and
+ *     must not be issued.  On the host the call holds the same lock as every
+ *     other entry point while it enqueues its work.
  *   - Always synchronous: the call waits for its stream and returns the
  *     device-side status (OC_ERR_NOT_SPD, OC_ERR_NONFINITE, ...), whatever
  *     oc_set_sync() says.

@@ -17,6 +17,17 @@
 // tcgen05.mma kind::tf32 M128 N128 K8 (12 per slice), warps 4..7 drain the
 // accumulator through swizzled 32x32 shared-memory boxes into TMA stores or
 // reduce-adds.  Triangular operands clip the k range of each tile.
+//
+// Segmented accumulation.  Adding an MMA's products into a TMEM accumulator
+// is not rounded to nearest: the sum is truncated, which biases every
+// addition towards zero by about half an ulp.  A chain of one accumulator
+// over a long k range (3 MMAs per 8-deep step) piles the bias up in
+// proportion to its length: measured against float64, the products with
+// k = 28672 came out about 6e-4 too small.  So each tile's k range is cut into
+// segments of KSEG; every segment restarts its accumulator (double-buffered in
+// TMEM, so the next segment's MMAs overlap), and the epilogue adds the
+// segments in fp32 registers, rounded to nearest, before the one store of
+// the tile.  The bias is then that of KSEG / 8 * 3 = 96 additions.
 #include <algorithm>
 
 #include "oc_internal.cuh"
@@ -26,6 +37,7 @@ namespace oc {
 namespace {
 
 constexpr int BM = 128, BN = 128, BK = 32;  // BK fp32 = 128 bytes = one swizzle row
+constexpr int KSEG = 256;                   // k per accumulator chain (a multiple of BK)
 constexpr int STAGES = 3;
 constexpr int TILE_BYTES = BM * BK * 4;      // 16 KB (A or B, one half)
 constexpr int STAGE_BYTES = 4 * TILE_BYTES;  // A_hi, A_lo, B_hi, B_lo
@@ -60,6 +72,9 @@ __device__ __forceinline__ void k_range(const Params& p, int i0, int j0, int& kb
   if (p.flags & kBUpper) ke = min(ke, j0 + BN);
   kb = (kb / BK) * BK;
 }
+
+// Segments of one tile's k range [kb, ke) (one, with no MMAs, when it is empty).
+__device__ __forceinline__ int n_segments(int kb, int ke) { return ke > kb ? (ke - kb + KSEG - 1) / KSEG : 1; }
 
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constant__ CUtensorMap mAl,
@@ -163,44 +178,48 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constan
       if (tile_skipped(p, i0, j0)) continue;
       int kb, ke;
       k_range(p, i0, j0, kb, ke);
-      const int acc = it & 1;
-      int w = 1;
-      if (lane == 0) w = mbar_wait(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1));
-      w = __shfl_sync(0xffffffffu, w, 0);
-      if (!w) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t dcol = tmem_base + static_cast<uint32_t>(acc * BN);
-      for (int k0 = kb; k0 < ke; k0 += BK) {
-        const int s = static_cast<int>(consumed % STAGES);
-        const uint32_t ph = static_cast<uint32_t>((consumed / STAGES) & 1);
-        w = 1;
-        if (lane == 0) w = mbar_wait(&full[s], ph) && !*abort_flag;
+      const int nseg = n_segments(kb, ke);
+      for (int sg = 0; sg < nseg && ok; ++sg) {
+        const int acc = it & 1;
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1));
         w = __shfl_sync(0xffffffffu, w, 0);
         if (!w) { ok = false; break; }
         tc_fence_after();
-        if (lane == 0) {
-          const uint32_t sa = smem_u32(stage_base + s * STAGE_BYTES);
-          const uint32_t sah = sa, sal = sa + TILE_BYTES, sbh = sa + 2 * TILE_BYTES, sbl = sa + 3 * TILE_BYTES;
+        const uint32_t dcol = tmem_base + static_cast<uint32_t>(acc * BN);
+        const int s0 = kb + sg * KSEG, s1 = min(ke, s0 + KSEG);
+        for (int k0 = s0; k0 < s1; k0 += BK) {
+          const int s = static_cast<int>(consumed % STAGES);
+          const uint32_t ph = static_cast<uint32_t>((consumed / STAGES) & 1);
+          w = 1;
+          if (lane == 0) w = mbar_wait(&full[s], ph) && !*abort_flag;
+          w = __shfl_sync(0xffffffffu, w, 0);
+          if (!w) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sa = smem_u32(stage_base + s * STAGE_BYTES);
+            const uint32_t sah = sa, sal = sa + TILE_BYTES, sbh = sa + 2 * TILE_BYTES, sbl = sa + 3 * TILE_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 8; ++kk) {
-            const uint64_t ah = smem_desc_sw128(sah + kk * 32, 16, 1024);
-            const uint64_t al = smem_desc_sw128(sal + kk * 32, 16, 1024);
-            const uint64_t bh = smem_desc_sw128(sbh + kk * 32, 16, 1024);
-            const uint64_t bl = smem_desc_sw128(sbl + kk * 32, 16, 1024);
-            const uint32_t first = (k0 == kb && kk == 0) ? 0u : 1u;
-            mma_tf32_ss(dcol, al, bh, idesc, first);
-            mma_tf32_ss(dcol, ah, bl, idesc, 1u);
-            mma_tf32_ss(dcol, ah, bh, idesc, 1u);
+            for (int kk = 0; kk < BK / 8; ++kk) {
+              const uint64_t ah = smem_desc_sw128(sah + kk * 32, 16, 1024);
+              const uint64_t al = smem_desc_sw128(sal + kk * 32, 16, 1024);
+              const uint64_t bh = smem_desc_sw128(sbh + kk * 32, 16, 1024);
+              const uint64_t bl = smem_desc_sw128(sbl + kk * 32, 16, 1024);
+              const uint32_t first = (k0 == s0 && kk == 0) ? 0u : 1u;
+              mma_tf32_ss(dcol, al, bh, idesc, first);
+              mma_tf32_ss(dcol, ah, bl, idesc, 1u);
+              mma_tf32_ss(dcol, ah, bh, idesc, 1u);
+            }
+            mma_commit(&empty[s]);
           }
-          mma_commit(&empty[s]);
+          __syncwarp();
+          ++consumed;
         }
+        if (!ok) break;
+        if (lane == 0) mma_commit(&tfull[acc]);
         __syncwarp();
-        ++consumed;
+        ++it;
       }
-      if (!ok) break;
-      if (lane == 0) mma_commit(&tfull[acc]);
-      __syncwarp();
-      ++it;
     }
     if (lane == 0) {
       if (!ok) {
@@ -217,40 +236,55 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constan
     unsigned char* stage_buf = epi_base + q * 2 * EPI_BOX_BYTES;
     int it = 0, nbuf = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
       const int i0 = (t % p.tiles_m) * BM, j0 = (t / p.tiles_m) * BN;
       if (tile_skipped(p, i0, j0)) continue;
       int kb, ke;
       k_range(p, i0, j0, kb, ke);
       const bool empty_k = kb >= ke;
-      const int acc = it & 1;
-      int w = 1;
-      if (lane == 0) w = mbar_wait(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1)) && !*abort_flag;
-      w = __shfl_sync(0xffffffffu, w, 0);
-      if (!w) { ok = false; break; }
-      tc_fence_after();
-      if (!(empty_k && p.accumulate)) {
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          if (!empty_k) {
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
-                                   static_cast<uint32_t>(acc * BN + c * 32);
+      const int nseg = n_segments(kb, ke);
+      // row `lane` of this warp's 32 rows, all BN columns: the tile's sum
+      float sum[BN];
+#pragma unroll
+      for (int e = 0; e < BN; ++e) sum[e] = 0.f;
+      for (int sg = 0; sg < nseg; ++sg) {
+        const int acc = it & 1;
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1)) && !*abort_flag;
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) { ok = false; break; }
+        tc_fence_after();
+        if (!empty_k) {
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            const uint32_t taddr =
+                tmem_base + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(acc * BN + c * 32);
             tmem_ld_32x32b_x32(taddr, r);
             tmem_ld_wait();
-          } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = 0u;
+            for (int e = 0; e < 32; ++e) sum[32 * c + e] += __uint_as_float(r[e]);
           }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        ++it;
+      }
+      if (!ok) break;
+      if (!(empty_k && p.accumulate)) {
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
           unsigned char* buf = stage_buf + (nbuf & 1) * EPI_BOX_BYTES;
           if (lane == 0) bulk_wait_group_read<1>();
           __syncwarp();
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             float4 v;
-            v.x = __uint_as_float(r[4 * k + 0]) * p.alpha;
-            v.y = __uint_as_float(r[4 * k + 1]) * p.alpha;
-            v.z = __uint_as_float(r[4 * k + 2]) * p.alpha;
-            v.w = __uint_as_float(r[4 * k + 3]) * p.alpha;
+            v.x = sum[32 * c + 4 * k + 0] * p.alpha;
+            v.y = sum[32 * c + 4 * k + 1] * p.alpha;
+            v.z = sum[32 * c + 4 * k + 2] * p.alpha;
+            v.w = sum[32 * c + 4 * k + 3] * p.alpha;
             *reinterpret_cast<float4*>(buf + lane * 128 + ((k ^ (lane & 7)) << 4)) = v;
           }
           fence_proxy_async_smem();
@@ -263,10 +297,6 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constan
           ++nbuf;
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
-      ++it;
     }
     if (!ok && lane == 0) {
       record_error(p.status, kDevTimeout);
@@ -291,6 +321,9 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constan
 // per slice as the single-CTA kernel for twice the MMA work.  Both producers
 // arm the leader's "full" barrier with their own bytes; the leader issues
 // M=256 N=256 K=8 kind::tf32 MMAs (3 per k step) and commits to both CTAs.
+// Segmented accumulation as above; the tile's running sum (256 columns per
+// row) is held by eight epilogue warps, 128 columns each: warps 4..11, warp w
+// reading TMEM lanes 32 (w % 4) .. + 31 and column half (w - 4) / 4.
 constexpr int PM = 256, PN = 256;              // pair tile
 constexpr int P_STAGES = 3;
 constexpr int P_STAGE_BYTES = 4 * TILE_BYTES;  // A_hi, A_lo, B_hi, B_lo (128 rows each)
@@ -298,6 +331,9 @@ constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + EPI_BYTES + 1024 + 1024;
 static_assert(P_SMEM_BYTES <= 232448, "shared memory per CTA");
 constexpr uint32_t P_TMEM_COLS = 512;
 constexpr uint16_t kPairMask = 0x3;
+constexpr int P_THREADS = 384;
+constexpr int P_EPI_WARPS = 8;      // one 4 KB staging box each: P_EPI_WARPS * EPI_BOX_BYTES == EPI_BYTES
+static_assert(P_EPI_WARPS * EPI_BOX_BYTES == EPI_BYTES, "pair staging boxes");
 
 __device__ __forceinline__ bool pair_tile_skipped(const Params& p, int i0, int j0) {
   return (p.flags & kCLowerOnly) && j0 > i0 + PM - 1;
@@ -313,7 +349,7 @@ __device__ __forceinline__ void pair_k_range(const Params& p, int i0, int j0, in
   kb = (kb / BK) * BK;
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(P_THREADS, 1)
 gemm_tf32x3_pair_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constant__ CUtensorMap mAl,
                         const __grid_constant__ CUtensorMap mBh, const __grid_constant__ CUtensorMap mBl,
                         const __grid_constant__ CUtensorMap mC, const Params p) {
@@ -345,7 +381,7 @@ gemm_tf32x3_pair_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_co
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 2 * EPI_WARPS);
+      mbar_init(&tempty[a], 2 * P_EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -424,44 +460,48 @@ gemm_tf32x3_pair_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_co
         if (pair_tile_skipped(p, i0, j0)) continue;
         int kb, ke;
         pair_k_range(p, i0, j0, kb, ke);
-        const int acc = it & 1;
-        int w = 1;
-        if (lane == 0) w = mbar_wait(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1));
-        w = __shfl_sync(0xffffffffu, w, 0);
-        if (!w) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t dcol = tmem_base + static_cast<uint32_t>(acc * PN);
-        for (int k0 = kb; k0 < ke; k0 += BK) {
-          const int s = static_cast<int>(consumed % P_STAGES);
-          const uint32_t ph = static_cast<uint32_t>((consumed / P_STAGES) & 1);
-          w = 1;
-          if (lane == 0) w = mbar_wait(&full[s], ph) && !*abort_flag;
+        const int nseg = n_segments(kb, ke);
+        for (int sg = 0; sg < nseg && ok; ++sg) {
+          const int acc = it & 1;
+          int w = 1;
+          if (lane == 0) w = mbar_wait(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1));
           w = __shfl_sync(0xffffffffu, w, 0);
           if (!w) { ok = false; break; }
           tc_fence_after();
-          if (lane == 0) {
-            const uint32_t sa = smem_u32(stage_base + s * P_STAGE_BYTES);
-            const uint32_t sah = sa, sal = sa + TILE_BYTES, sbh = sa + 2 * TILE_BYTES, sbl = sa + 3 * TILE_BYTES;
+          const uint32_t dcol = tmem_base + static_cast<uint32_t>(acc * PN);
+          const int s0 = kb + sg * KSEG, s1 = min(ke, s0 + KSEG);
+          for (int k0 = s0; k0 < s1; k0 += BK) {
+            const int s = static_cast<int>(consumed % P_STAGES);
+            const uint32_t ph = static_cast<uint32_t>((consumed / P_STAGES) & 1);
+            w = 1;
+            if (lane == 0) w = mbar_wait(&full[s], ph) && !*abort_flag;
+            w = __shfl_sync(0xffffffffu, w, 0);
+            if (!w) { ok = false; break; }
+            tc_fence_after();
+            if (lane == 0) {
+              const uint32_t sa = smem_u32(stage_base + s * P_STAGE_BYTES);
+              const uint32_t sah = sa, sal = sa + TILE_BYTES, sbh = sa + 2 * TILE_BYTES, sbl = sa + 3 * TILE_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < BK / 8; ++kk) {
-              const uint64_t ah = smem_desc_sw128(sah + kk * 32, 16, 1024);
-              const uint64_t al = smem_desc_sw128(sal + kk * 32, 16, 1024);
-              const uint64_t bh = smem_desc_sw128(sbh + kk * 32, 16, 1024);
-              const uint64_t bl = smem_desc_sw128(sbl + kk * 32, 16, 1024);
-              const uint32_t first = (k0 == kb && kk == 0) ? 0u : 1u;
-              mma_tf32_ss_pair(dcol, al, bh, idesc, first);
-              mma_tf32_ss_pair(dcol, ah, bl, idesc, 1u);
-              mma_tf32_ss_pair(dcol, ah, bh, idesc, 1u);
+              for (int kk = 0; kk < BK / 8; ++kk) {
+                const uint64_t ah = smem_desc_sw128(sah + kk * 32, 16, 1024);
+                const uint64_t al = smem_desc_sw128(sal + kk * 32, 16, 1024);
+                const uint64_t bh = smem_desc_sw128(sbh + kk * 32, 16, 1024);
+                const uint64_t bl = smem_desc_sw128(sbl + kk * 32, 16, 1024);
+                const uint32_t first = (k0 == s0 && kk == 0) ? 0u : 1u;
+                mma_tf32_ss_pair(dcol, al, bh, idesc, first);
+                mma_tf32_ss_pair(dcol, ah, bl, idesc, 1u);
+                mma_tf32_ss_pair(dcol, ah, bh, idesc, 1u);
+              }
+              mma_commit_pair(&empty[s], kPairMask);
             }
-            mma_commit_pair(&empty[s], kPairMask);
+            __syncwarp();
+            ++consumed;
           }
+          if (!ok) break;
+          if (lane == 0) mma_commit_pair(&tfull[acc], kPairMask);
           __syncwarp();
-          ++consumed;
+          ++it;
         }
-        if (!ok) break;
-        if (lane == 0) mma_commit_pair(&tfull[acc], kPairMask);
-        __syncwarp();
-        ++it;
       }
       if (lane == 0) {
         if (!ok) {
@@ -477,62 +517,73 @@ gemm_tf32x3_pair_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_co
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp - 4;
-    unsigned char* stage_buf = epi_base + q * 2 * EPI_BOX_BYTES;
+    const int q = warp & 3;                 // TMEM lanes 32q .. 32q + 31
+    const int hc = (warp - 4) >> 2;         // columns 128 hc .. 128 hc + 127 of the tile
+    unsigned char* buf = epi_base + (warp - 4) * EPI_BOX_BYTES;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
-    int it = 0, nbuf = 0;
+    int it = 0;
     bool ok = true;
-    for (int t = cid; t < n_tiles; t += ncl) {
+    for (int t = cid; t < n_tiles && ok; t += ncl) {
       const int i0 = (t % p.tiles_m) * PM, j0 = (t / p.tiles_m) * PN;
       if (pair_tile_skipped(p, i0, j0)) continue;
       int kb, ke;
       pair_k_range(p, i0, j0, kb, ke);
       const bool empty_k = kb >= ke;
-      const int acc = it & 1;
-      int w = 1;
-      if (lane == 0) w = mbar_wait(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1)) && !*abort_flag;
-      w = __shfl_sync(0xffffffffu, w, 0);
-      if (!w) { ok = false; break; }
-      tc_fence_after();
-      if (!(empty_k && p.accumulate)) {
-        for (int c = 0; c < PN / 32; ++c) {
-          uint32_t r[32];
-          if (!empty_k) {
+      const int nseg = n_segments(kb, ke);
+      float sum[128];
+#pragma unroll
+      for (int e = 0; e < 128; ++e) sum[e] = 0.f;
+      for (int sg = 0; sg < nseg; ++sg) {
+        const int acc = it & 1;
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1)) && !*abort_flag;
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) { ok = false; break; }
+        tc_fence_after();
+        if (!empty_k) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
-                                   static_cast<uint32_t>(acc * PN + c * 32);
+                                   static_cast<uint32_t>(acc * PN + hc * 128 + c * 32);
             tmem_ld_32x32b_x32(taddr, r);
             tmem_ld_wait();
-          } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = 0u;
+            for (int e = 0; e < 32; ++e) sum[32 * c + e] += __uint_as_float(r[e]);
           }
-          unsigned char* buf = stage_buf + (nbuf & 1) * EPI_BOX_BYTES;
-          if (lane == 0) bulk_wait_group_read<1>();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+        ++it;
+      }
+      if (!ok) break;
+      if (!(empty_k && p.accumulate)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          // the store that last read the box must be done reading it
+          if (lane == 0) bulk_wait_group_read<0>();
           __syncwarp();
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             float4 v;
-            v.x = __uint_as_float(r[4 * k + 0]) * p.alpha;
-            v.y = __uint_as_float(r[4 * k + 1]) * p.alpha;
-            v.z = __uint_as_float(r[4 * k + 2]) * p.alpha;
-            v.w = __uint_as_float(r[4 * k + 3]) * p.alpha;
+            v.x = sum[32 * c + 4 * k + 0] * p.alpha;
+            v.y = sum[32 * c + 4 * k + 1] * p.alpha;
+            v.z = sum[32 * c + 4 * k + 2] * p.alpha;
+            v.w = sum[32 * c + 4 * k + 3] * p.alpha;
             *reinterpret_cast<float4*>(buf + lane * 128 + ((k ^ (lane & 7)) << 4)) = v;
           }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (p.accumulate) tma_reduce_add_2d(&mC, buf, j0 + c * 32, i0 + half + 32 * q);
-            else tma_store_2d(&mC, buf, j0 + c * 32, i0 + half + 32 * q);
+            const int col = j0 + hc * 128 + c * 32, row = i0 + half + 32 * q;
+            if (p.accumulate) tma_reduce_add_2d(&mC, buf, col, row);
+            else tma_store_2d(&mC, buf, col, row);
             bulk_commit_group();
           }
-          ++nbuf;
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
-      ++it;
     }
     if (!ok && lane == 0) {
       record_error(p.status, kDevTimeout);
@@ -738,7 +789,7 @@ void gemm_tf32x3(const Ctx& c, int64_t M, int64_t N, int64_t K, float alpha, con
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.blockDim = dim3(P_THREADS, 1, 1);
     cfg.dynamicSmemBytes = P_SMEM_BYTES;
     cfg.stream = c.stream;
     cfg.attrs = attr;

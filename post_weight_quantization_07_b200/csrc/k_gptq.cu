@@ -330,16 +330,6 @@ __global__ void pack_kernel(const unsigned char* __restrict__ codes8, int64_t m,
   out[e] = word;
 }
 
-// D = -H/2 = -Xhat^T Xhat: the starting value of the QEP cross term, onto
-// which the cross product adds X^T Xhat.  count4 float4 elements.
-__global__ void neg_half_kernel(const float4* __restrict__ H, float4* __restrict__ D, int64_t count4) {
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < count4;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float4 h = H[e];
-    D[e] = make_float4(-0.5f * h.x, -0.5f * h.y, -0.5f * h.z, -0.5f * h.w);
-  }
-}
-
 __global__ void copy_kernel(const float* __restrict__ a, float* __restrict__ b, int64_t count) {
   const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (e < count) b[e] = a[e];
@@ -434,14 +424,6 @@ void launch_pack(const Ctx& c, const unsigned char* codes8, int64_t m, int64_t n
 void launch_invert_perm(const Ctx& c, int32_t* perm2, int64_t n) {
   invert_perm_kernel<<<blocks_for(n, 256), 256, 0, c.stream>>>(perm2, n, perm2 + n);
   check_launch("invert_perm_kernel");
-}
-
-void launch_neg_half(const Ctx& c, const float* H, float* D, int64_t n) {
-  const int64_t count4 = n * n / 4;  // n is a multiple of 64
-  const int grid = static_cast<int>(std::min<int64_t>(blocks_for(count4, 256), static_cast<int64_t>(c.sm_count) * 8));
-  neg_half_kernel<<<grid, 256, 0, c.stream>>>(reinterpret_cast<const float4*>(H), reinterpret_cast<float4*>(D),
-                                              count4);
-  check_launch("neg_half_kernel");
 }
 
 void launch_copy_f32(const Ctx& c, const float* src, float* dst, int64_t count) {

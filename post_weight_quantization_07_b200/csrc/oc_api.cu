@@ -147,6 +147,8 @@ void fail(int status, const char* fmt, ...) {
 
 void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
 
+std::mutex& library_mutex() { return g_mu; }
+
 void check_cuda(cudaError_t e, const char* what) {
   if (e != cudaSuccess) fail(OC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
@@ -296,6 +298,8 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
   sizing.take<unsigned char>(n);          // dead-column mask
   sizing.take<float>(factor_split_floats(n));
   sizing.take<DiagStats>(1);
+  const size_t cross_bytes = terms_given ? 0 : cross_scratch_bytes(n_tok, n);
+  sizing.take<unsigned char>(cross_bytes);  // the cross product's operands
   Carve cv{workspace(c, sizing.off + 256)};
   float* D = cv.take<float>(nn);
   float* Xi = cv.take<float>(nn);
@@ -314,6 +318,7 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
   unsigned char* dead = cv.take<unsigned char>(n);
   float* fsplit = cv.take<float>(factor_split_floats(n));
   DiagStats* stats = cv.take<DiagStats>(1);
+  unsigned char* cross_scratch = cv.take<unsigned char>(cross_bytes);
   auto Gl = [&](int l) { return Gs + static_cast<size_t>(l) * mn; };
   const size_t nn_bytes = nn * sizeof(float);
 
@@ -324,7 +329,7 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
     }
     {
       PhaseScope ps(c, kPhHessian);
-      launch_atb_bf16(c, Xhat, Xhat, n_tok, n, n, 2.0f, H, n, true);
+      launch_atb16(c, Xhat, Xhat, n_tok, n, n, 2.0f, H, n, true);
     }
     {
       PhaseScope ps(c, kPhHessianFix);
@@ -360,26 +365,13 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
     check_cuda(cudaMemcpyAsync(D, D_in, nn_bytes, cudaMemcpyDeviceToDevice, c.stream), "copy d");
   } else {
     {
-      // d = X^T Xhat - Xhat^T Xhat: start from -H/2 and add the cross product
-      PhaseScope ps(c, kPhQepCrossFix);
-      launch_neg_half(c, H, D, n);
-    }
-    {
+      // d = (X - Xhat)^T Xhat in token ranges: between two launches the
+      // high-priority factorisation can take the freed SMs for its wide
+      // tensor-core products
       PhaseScope ps(c, kPhQepCross);
-      if (shared_factor) {
-        // In token ranges: between two launches the high-priority factorisation
-        // can take the freed SMs for its wide tensor-core products.
-        const int64_t parts = std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens));
-        const int64_t per = ((n_tok + parts - 1) / parts + 63) / 64 * 64;
-        const unsigned char* xb = static_cast<const unsigned char*>(X);
-        const unsigned char* hb = static_cast<const unsigned char*>(Xhat);
-        for (int64_t t0 = 0; t0 < n_tok; t0 += per) {
-          const int64_t len = std::min(per, n_tok - t0);
-          launch_atb_bf16(c, xb + t0 * n * 2, hb + t0 * n * 2, len, n, n, 1.0f, D, n, false, c.sm_count - kSideSMs);
-        }
-      } else {
-        launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D, n, false, 0);
-      }
+      const int parts = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens)));
+      launch_cross_product(c, X, Xhat, n_tok, n, H, D, cross_scratch, parts,
+                           shared_factor ? c.sm_count - kSideSMs : 0);
     }
   }
   {
@@ -546,7 +538,7 @@ int oc_hessian_accumulate(const void* X, int64_t n_tok, int64_t n, float* H, voi
     Ctx c = make_ctx(stream);
     {
       PhaseScope ps(c, kPhHessian);
-      launch_atb_bf16(c, X, X, n_tok, n, n, 2.0f, H, n, true);
+      launch_atb16(c, X, X, n_tok, n, n, 2.0f, H, n, true);
     }
     {
       PhaseScope ps(c, kPhHessianFix);
@@ -587,6 +579,8 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
     sizing.take<float>(nn + 4096);                // recursion scratch of the side-stream factorisation
     sizing.take<float>(factor_split_floats(n));   // split copies inside the factorisation
     sizing.take<DiagStats>(1);
+    const size_t cross_bytes = cross_scratch_bytes(n_tok, n);
+    sizing.take<unsigned char>(cross_bytes);      // the cross product's operands
     Carve cv{workspace(c, sizing.off + 256)};
     float* D = cv.take<float>(nn);
     float* Hs = H_opt ? nullptr : cv.take<float>(nn);
@@ -600,13 +594,13 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
     float* Fs = cv.take<float>(nn + 4096);
     float* fsplit = cv.take<float>(factor_split_floats(n));
     DiagStats* stats = cv.take<DiagStats>(1);
+    unsigned char* cross_scratch = cv.take<unsigned char>(cross_bytes);
 
-    // d = X^T Xhat - Xhat^T Xhat  (the second term from H = 2 Xhat^T Xhat)
     const float* Hp = H_opt;
     if (!H_opt) {
       PhaseScope ps(c, kPhQepSyrk);
       check_cuda(cudaMemsetAsync(Hs, 0, nn * sizeof(float), c.stream), "memset Hs");
-      launch_atb_bf16(c, Xhat, Xhat, n_tok, n, n, 2.0f, Hs, n, true);
+      launch_atb16(c, Xhat, Xhat, n_tok, n, n, 2.0f, Hs, n, true);
       launch_mirror_upper(c, Hs, n);
       Hp = Hs;
     }
@@ -628,19 +622,10 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
     }
     check_cuda(cudaEventRecord(ss.join, cs.stream), "cudaEventRecord(join)");
     {
-      PhaseScope ps(c, kPhQepCrossFix);
-      launch_neg_half(c, Hp, D, n);
-    }
-    {
+      // d = (X - Xhat)^T Xhat, in token ranges beside the factorisation
       PhaseScope ps(c, kPhQepCross);
-      const int64_t parts = std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens));
-      const int64_t per = ((n_tok + parts - 1) / parts + 63) / 64 * 64;
-      const unsigned char* xb = static_cast<const unsigned char*>(X);
-      const unsigned char* hb = static_cast<const unsigned char*>(Xhat);
-      for (int64_t t0 = 0; t0 < n_tok; t0 += per) {
-        const int64_t len = std::min(per, n_tok - t0);
-        launch_atb_bf16(c, xb + t0 * n * 2, hb + t0 * n * 2, len, n, n, 1.0f, D, n, false, c.sm_count - kSideSMs);
-      }
+      const int parts = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens)));
+      launch_cross_product(c, X, Xhat, n_tok, n, Hp, D, cross_scratch, parts, c.sm_count - kSideSMs);
     }
     {
       // G = W d on the tensor cores (3xTF32 from split operands)
@@ -884,21 +869,20 @@ int oc_qep_terms(const void* X, const void* Xhat, int64_t n_tok, int64_t n, floa
       if (n_tok == 0) check_cuda(cudaMemsetAsync(D_part, 0, nn_bytes, c.stream), "memset D_part");
     }
     if (n_tok == 0) return finish(c);
+    unsigned char* cross_scratch = reinterpret_cast<unsigned char*>(workspace(c, cross_scratch_bytes(n_tok, n) + 256));
     {
       PhaseScope ps(c, kPhHessian);
-      launch_atb_bf16(c, Xhat, Xhat, n_tok, n, n, 2.0f, H_part, n, true);
+      launch_atb16(c, Xhat, Xhat, n_tok, n, n, 2.0f, H_part, n, true);
     }
     {
       PhaseScope ps(c, kPhHessianFix);
       launch_mirror_upper(c, H_part, n);
     }
     {
-      PhaseScope ps(c, kPhQepCrossFix);
-      launch_neg_half(c, H_part, D_part, n);
-    }
-    {
+      // D_part = (X - Xhat)^T Xhat
       PhaseScope ps(c, kPhQepCross);
-      launch_atb_bf16(c, X, Xhat, n_tok, n, n, 1.0f, D_part, n, false);
+      const int parts = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens)));
+      launch_cross_product(c, X, Xhat, n_tok, n, H_part, D_part, cross_scratch, parts, 0);
     }
     return finish(c);
   });

@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -40,6 +41,9 @@ struct Failure {
 [[noreturn]] void fail(int status, const char* fmt, ...);
 void check_cuda(cudaError_t e, const char* what);
 void set_last_error(const char* msg);  // text returned by oc_last_error() on this thread
+// The lock every entry point holds while it sets up and enqueues its work
+// (launch helpers share host-side state such as one-time attribute flags).
+std::mutex& library_mutex();
 void check_launch(const char* kernel);
 
 // ------------------------------------------------------------------ profiling
@@ -55,10 +59,11 @@ enum Phase : int {
   kPhGptqTrailing,  // trailing updates of later columns
   kPhGptqPack,      // inverse permutation + bit packing
   kPhHessianFix,    // clearing H, mirroring its upper triangle
-  kPhQepCrossFix,   // clearing d, subtracting Xhat^T Xhat
+  kPhQepCrossFix,   // clearing d before the cross product accumulates into it
   kPhRotate,        // Hadamard rotation
   kPhLpcdLeft,      // LPCD's relaxed layer-1 step (products, factorisation, solve)
   kPhGemv,          // dequantising GEMV over packed codes
+  kPhQepDiff,       // cross-product operands when no Hessian launch carries them
   kNumPhases
 };
 
@@ -101,8 +106,18 @@ CUtensorMap make_tmap_2d(const void* base, CUtensorMapDataType dt, int elem_byte
 // [n_tok x M] and [n_tok x N]; C fp32 [M x N] (ldc).  upper_only: A == B and
 // only tiles touching the upper triangle are computed (the caller mirrors).
 // max_ctas > 0 caps the persistent grid (leaving SMs free for concurrent work).
-void launch_atb_bf16(const Ctx& c, const void* A, const void* B, int64_t n_tok, int64_t M,
-                     int64_t N, float alpha, float* C, int64_t ldc, bool upper_only, int max_ctas = 0);
+void launch_atb16(const Ctx& c, const void* A, const void* B, int64_t n_tok, int64_t M, int64_t N, float alpha,
+                  float* C, int64_t ldc, bool upper_only, int max_ctas = 0);
+
+// QEP's cross term d = (X - Xhat)^T Xhat (n x n, fp32, overwritten) from the
+// bf16 token-major pair X, Xhat [n_tok x n] and H = 2 Xhat^T Xhat of the same
+// tokens (its diagonal sets per-feature fp16 scales).  Runs as `parts` token
+// slices on at most max_ctas SMs (0: all), each slice's operands prepared
+// while the previous slice runs.  `scratch`: cross_scratch_bytes(n_tok, n)
+// bytes of device memory, 256-byte aligned.
+size_t cross_scratch_bytes(int64_t n_tok, int64_t n);
+void launch_cross_product(const Ctx& c, const void* X, const void* Xhat, int64_t n_tok, int64_t n, const float* H,
+                          float* d, void* scratch, int parts, int max_ctas);
 
 // Per-device side stream and fork/join events for running the (latency
 // bound) factorisation beside a tensor-core product on the call's stream.
@@ -207,7 +222,6 @@ void launch_pack(const Ctx& c, const unsigned char* codes8, int64_t m, int64_t n
 void launch_invert_perm(const Ctx& c, int32_t* perm2, int64_t n);
 
 // QEP pieces.
-void launch_neg_half(const Ctx& c, const float* H, float* D, int64_t n);  // D = -H/2
 void launch_copy_f32(const Ctx& c, const float* src, float* dst, int64_t count);
 void launch_fill_f32(const Ctx& c, float* dst, int64_t count, float v);
 void launch_check_finite(const Ctx& c, const float* x, int64_t count);

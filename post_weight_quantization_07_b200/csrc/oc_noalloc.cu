@@ -16,6 +16,8 @@
 #include <cstdio>
 #include <mutex>
 
+#include <cuda.h>
+
 #include "oc_internal.cuh"
 
 namespace oc {
@@ -29,21 +31,55 @@ constexpr size_t kNoallocBytes = size_t(6) << 20;  // 6 MiB
 // address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocBytes];
 
-std::mutex g_setup_mu;
-void* g_scratch_addr[64] = {};
+// Device address of g_noalloc_scratch per device, with the id of the context
+// it was looked up in: a process that destroys a device's primary context
+// (cudaDeviceReset) and creates a new one gets the array at a new address.
+struct ScratchAddr {
+  unsigned long long ctx_id = 0;
+  void* addr = nullptr;
+};
+ScratchAddr g_scratch_addr[64];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <class Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  check_cuda(cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q), "cudaGetDriverEntryPoint");
+  if (q != cudaDriverEntryPointSuccess || p == nullptr) fail(OC_ERR_UNSUPPORTED, "driver does not provide %s", name);
+  return reinterpret_cast<Fn>(p);
+}
+
+// Id of the context current on this thread (the device's primary context,
+// made current by the runtime's cudaGetDevice/cudaFree-free calls before).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) fail(OC_ERR_CUDA, "no current CUDA context");
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) fail(OC_ERR_CUDA, "cuCtxGetId failed");
+  return id;
+}
 
 // Device address of g_noalloc_scratch on `dev` (which must be current),
-// looked up once per device on the first call there.
+// looked up on the first call there and again only if the context changed.
 unsigned char* scratch_address(int dev) {
-  std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  // the runtime makes the device's primary context current (no allocation)
+  check_cuda(cudaSetDevice(dev), "cudaSetDevice");
+  const unsigned long long id = current_context_id();
+  ScratchAddr& s = g_scratch_addr[dev];
+  if (s.addr == nullptr || s.ctx_id != id) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr)
       fail(OC_ERR_CUDA, "cudaGetSymbolAddress(g_noalloc_scratch) failed: %s", cudaGetErrorString(e));
-    g_scratch_addr[dev] = p;
+    s.addr = p;
+    s.ctx_id = id;
   }
-  return static_cast<unsigned char*>(g_scratch_addr[dev]);
+  return static_cast<unsigned char*>(s.addr);
 }
 
 // Same 256-byte-aligned carving as the allocating entry point, over a fixed base.
@@ -164,6 +200,9 @@ extern "C" int oc_gptq_quantize_noalloc(const float* W, int64_t m, int64_t n, co
                                         float* scales, float* zeros, int32_t* perm_out, void* stream) {
   try {
     oc::set_last_error("");
+    // the same lock as every other entry point: the launch helpers share
+    // host-side state (one-time kernel attribute flags, the launch counter)
+    std::lock_guard<std::mutex> lock(oc::library_mutex());
     return oc::run(W, m, n, H, wbits, groupsize, damp, act_order, codes, scales, zeros, perm_out, stream);
   } catch (const oc::Failure& e) {
     oc::set_last_error(e.msg);

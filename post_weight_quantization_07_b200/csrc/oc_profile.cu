@@ -24,7 +24,7 @@ std::atomic<int64_t> g_launches{0};
 const char* const kPhaseNames[kNumPhases] = {
     "hessian_syrk", "qep_cross", "qep_syrk", "qep_w_delta", "factor",
     "qep_apply", "gptq_prep", "gptq_sweep", "gptq_trailing", "gptq_pack",
-    "hessian_fixup", "qep_cross_fixup", "hadamard_rotate", "lpcd_left_project", "dequant_gemv"};
+    "hessian_fixup", "qep_cross_fixup", "hadamard_rotate", "lpcd_left_project", "dequant_gemv", "qep_diff"};
 
 cudaEvent_t take_event() {
   if (!g_pool.empty()) {

@@ -12,8 +12,11 @@ Tolerances (the quantisation workload's stated bars):
   scales / zeros    relative error <= 1e-5 (zeros: equal unless -min/scale sits
                     within 1e-3 of a rounding boundary);
   layer error       ||(W - Q) X^T||_F within 1% of the oracle's.
-QEP output: max |W'_gpu - W'_oracle| <= 1e-5 * max |W| (derived in the design
-notes from the fp32 arithmetic of the path).
+QEP output: max |W'_gpu - W'_oracle| <= 1e-5 * max |W|.  The library forms the
+cross term from D = bf16(X - Xhat), each difference rounded once (relative
+error <= 2^-9, of random sign), so the correction W' - W carries about 1e-3 of
+its own size from that rounding, plus fp32 accumulation and the fp32 factor;
+on these layers the correction is a few percent of W at most.
 """
 import numpy as np
 import pytest
@@ -98,6 +101,49 @@ def test_qep_matches_oracle(use_h, shape):
     assert err <= QEP_TOL * np.abs(W).max(), (err, corr)
     # the correction itself is reproduced to a small fraction of its size
     assert np.abs((Wg - W) - (Wo - W)).max() <= 2e-3 * corr
+
+
+def _large_channel(X, Xh, channel=5):
+    # one channel scaled by 2^15 (exact in bf16): its values pass fp16's
+    # largest finite 65504, which the per-feature scales of the cross
+    # product's fp16 operands must absorb
+    X, Xh = X.copy(), Xh.copy()
+    X[:, channel] *= 32768.0
+    Xh[:, channel] *= 32768.0
+    assert np.abs(Xh).max() > 65504.0
+    return X, Xh
+
+
+def _far_difference(X, Xh, channel=5, token=17):
+    # one value of X far from Xhat's: X - Xhat there exceeds 4 times the
+    # column's norm sqrt(sum_t Xhat^2), beyond what the fp16 scale taken from
+    # the Hessian diagonal allows, so the cross product must take its bf16 path
+    X = X.copy()
+    r = float(np.sqrt(np.sum(Xh[:, channel].astype(np.float64) ** 2)))
+    X[token, channel] = oracle._bf16(np.array([Xh[token, channel] + 64.0 * r]))[0]
+    return X, Xh
+
+
+@pytest.mark.parametrize("use_h", [False, True])
+@pytest.mark.parametrize("case", ["large_channel", "far_difference"])
+def test_qep_cross_operands_outside_fp16_range(use_h, case):
+    W, X, Xh = _qep_case(n=256, m=96, n_tok=3000, seed=19)
+    X, Xh = (_large_channel if case == "large_channel" else _far_difference)(X, Xh)
+    Ho = oracle.hessian(Xh)
+    Wo = oracle.qep_correct(W, X, Xh, 0.5, 0.01, H=Ho)
+    Hg = dev(gpu_hessian(Xh)) if use_h else None
+    Wg = oc.oc_qep_correct(dev(W), bf16_dev(X), bf16_dev(Xh), 0.5, 0.01, H_opt=Hg).cpu().numpy()
+    assert np.all(np.isfinite(Wg))
+    E, corr = Wg - Wo, Wo - W
+    if case == "large_channel":
+        # scaled fp16 operands: D to 11 significant bits
+        assert np.abs(E).max() <= QEP_TOL * np.abs(W).max()
+        assert np.linalg.norm(E) <= 2e-3 * np.linalg.norm(corr), np.linalg.norm(E) / np.linalg.norm(corr)
+    else:
+        # bf16 operands: D to 8 significant bits, about 1e-3 of the correction,
+        # which the planted difference makes as large as W itself
+        assert np.abs(E).max() <= 5e-3 * np.abs(corr).max(), np.abs(E).max() / np.abs(corr).max()
+        assert np.linalg.norm(E) <= 5e-3 * np.linalg.norm(corr), np.linalg.norm(E) / np.linalg.norm(corr)
 
 
 def test_qep_alpha_zero_is_identity_bitwise():
@@ -290,18 +336,21 @@ def test_end_to_end_512_workload():
 
 # ----------------------------------------------------------------------------- fused layer call
 
-@pytest.mark.parametrize("m,n,n_tok,wbits,G,act,dead", [
-    (512, 512, 2048, 4, 128, False, False),
-    (256, 384, 1500, 3, 64, True, False),
-    (96, 256, 1024, 4, 64, True, True),     # dead columns: two factorisations
-    (128, 1024, 4096, 2, 64, True, False),  # large enough for tensor-core factor nodes
+@pytest.mark.parametrize("m,n,n_tok,wbits,G,act,dead,big", [
+    (512, 512, 2048, 4, 128, False, False, False),
+    (256, 384, 1500, 3, 64, True, False, False),
+    (96, 256, 1024, 4, 64, True, True, False),     # dead columns: two factorisations
+    (128, 1024, 4096, 2, 64, True, False, False),  # large enough for tensor-core factor nodes
+    (160, 256, 1500, 4, 64, False, False, True),   # a difference beyond fp16's scaled range: bf16 cross product
 ])
-def test_fused_layer_matches_oracle(m, n, n_tok, wbits, G, act, dead):
+def test_fused_layer_matches_oracle(m, n, n_tok, wbits, G, act, dead, big):
     L = random_layer_host(m, n, n_tok, seed=3000 + n + m)
     W, X, Xh = L["W"].astype(np.float64), L["X"].copy(), L["Xhat"].copy()
     if dead:
         X[:, [7, 100]] = 0.0
         Xh[:, [7, 100]] = 0.0
+    if big:
+        X, Xh = _far_difference(X, Xh)
     Ho = oracle.hessian(Xh)
     Wpo = oracle.qep_correct(W, X, Xh, 0.5, 0.01, H=Ho)
     ref = oracle.gptq_quantize(Wpo, Ho, wbits, G, 0.01, act)
@@ -311,7 +360,16 @@ def test_fused_layer_matches_oracle(m, n, n_tok, wbits, G, act, dead):
     torch.cuda.synchronize()
     assert rel_fro(Hg.cpu().numpy(), Ho) <= H_TOL
     Wpg = Wpg.cpu().numpy()
-    assert np.abs(Wpg - Wpo).max() <= QEP_TOL * np.abs(W).max()
+    if big:
+        # bf16 cross-product operands on a correction as large as W itself:
+        # W' to about 1e-3 of the correction, and GPTQ judged on the GPU's
+        # own W' (a difference of that size moves group ranges by more than
+        # the scale tolerance)
+        assert np.abs(Wpg - Wpo).max() <= 5e-3 * np.abs(Wpo - W).max()
+        Wpo = Wpg.astype(np.float64)
+        ref = oracle.gptq_quantize(Wpo, Ho, wbits, G, 0.01, act)
+    else:
+        assert np.abs(Wpg - Wpo).max() <= QEP_TOL * np.abs(W).max()
     cg = oracle.unpack_codes(codes.cpu().numpy().view(np.uint32), wbits, n)
     sg, zg = scales.cpu().numpy(), zeros.cpu().numpy()
     pg = perm.cpu().numpy()

@@ -6,9 +6,11 @@ caching allocator, a service held to a fixed pre-reserved budget): it runs the
 same kernels as oc_gptq_quantize with all scratch taken from an array built
 into the library.  These tests call both through the C ABI with raw pointers
 and require the same results, within the tolerances of the other GPTQ parity
-tests, on two calls in a row (the second one finds the previous call's data
-left in the shared scratch).  The file sorts last so that a run stopping at
-the first failure has already run every other test.
+tests, on two calls in a row; a call on the same shape after a call on other
+data (which leaves its intermediates in the shared scratch at the same
+offsets) must repeat its results bit for bit and pass the oracle's replay.
+The file sorts last so that a run stopping at the first failure has already
+run every other test.
 """
 import ctypes
 
@@ -100,3 +102,29 @@ def test_noalloc_rejects_layers_beyond_its_scratch():
                  ctypes.c_void_p(s.data_ptr()), None, None)
     assert st == oc.OC_ERR_INVALID_ARG
     assert "scratch" in oc.oc_last_error()
+
+
+def test_noalloc_same_shape_repeat_and_oracle():
+    # Same shape three times: data A, data B, data A again.  The third call
+    # finds B's intermediates in the shared scratch at the very offsets it
+    # uses, and must still give A's results bit for bit; A's results must also
+    # pass the oracle's teacher-forced replay.
+    noalloc, _ = _bind()
+    m, n, wbits, G, act = 256, 512, 4, 128, True
+    Wa, Ha = _layer(m, n, 61)
+    Wb, Hb = _layer(m, n, 62)
+    first = _call(noalloc, Wa, Ha, wbits, G, 0.01, act)
+    other = _call(noalloc, Wb, Hb, wbits, G, 0.01, act)
+    again = _call(noalloc, Wa, Ha, wbits, G, 0.01, act)
+    for x, y in zip(first, again):
+        assert np.array_equal(x, y)
+    assert not np.array_equal(first[1], other[1])
+    codes, scales, zeros, perm = first
+    W64, H64 = Wa.cpu().numpy().astype(np.float64), Ha.cpu().numpy().astype(np.float64)
+    cg = oracle.unpack_codes(codes.view(np.uint32), wbits, n)
+    st = oracle.teacher_forced_check(W64, H64, wbits, G, 0.01, act, cg, scales, zeros, perm=perm)
+    assert st["n_bad"] == 0 and st["zero_bad"] == 0, st
+    assert st["scale_max_rel"] <= SCALE_TOL, st
+    ref = oracle.gptq_quantize(W64, H64, wbits, G, 0.01, act)
+    assert np.array_equal(perm, ref["perm"])
+    assert np.mean(cg == ref["codes"]) >= 0.99
