@@ -38,11 +38,13 @@ SM_COUNT = 148
 L2_BYTES = 126 * 1024 * 1024
 CPU_SAMPLE_TOKENS = 16384
 CPU_SAMPLE_ROWS = 2048
-# DRAM bytes (read + written) per launch of atb_bf16_kernel, the mean of its
-# two launches in one layer, from one ncu capture of dram__bytes_read.sum and
-# dram__bytes_write.sum on this workload at full size (profiles/ has the
-# summary and the command): 33 launches per layer, 20.4 GB in all.
-TRAFFIC_PER_LAUNCH = {"q_proj_4096": 617853192}
+# The recorded DRAM traffic of the dominant kernel: dram__bytes_read.sum +
+# dram__bytes_write.sum per launch from one ncu capture of a smaller case of the
+# same workload, scaled to a full-size launch, with the SHA-256 of the kernel's
+# source at capture time.  If the source has changed since, the traffic is
+# reported as null.
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "atb16_q_proj_4096_traffic.json")
+KERNEL_SOURCE = os.path.join(ROOT, "post_weight_quantization_07_b200", "csrc", "k_atb16.cu")
 
 
 def load_peaks():
@@ -226,16 +228,40 @@ def phase_work(spec, factorisations=1):
         "gptq_pack": (m * n + m * n * spec.wbits // 8 + m * (n // G) * 8, "byte", "hbm"),
         # clear H (4n^2 written), mirror the upper triangle (2n^2 read + 2n^2 written)
         "hessian_fixup": (8 * n * n, "byte", "hbm"),
-        # clear d (4n^2), then d -= H/2 (read d and H, write d)
-        "qep_cross_fixup": (16 * n * n, "byte", "hbm"),
         # W (fp32), X and Xhat (bf16) read and written once each
         "hadamard_rotate": (2 * (4 * m * n + 2 * 2 * N * n), "byte", "hbm"),
     }
 
 
-def f32_simt_peak_tflops(sm_mhz):
-    # 148 SMs x 128 fp32 lanes x 2 flop per FMA x clock
-    return SM_COUNT * 128 * 2 * sm_mhz * 1e6 / 1e12
+def cross_slices(spec):
+    """Token slices the library runs the QEP cross product in (one launch of
+    the product each): 8192 tokens or more per slice, at most 32."""
+    return max(1, min(32, spec.n_tok // 8192))
+
+
+def gemm_bytes(spec):
+    """Algorithmic DRAM bytes of the two bf16-input phases of one layer: X and
+    Xhat read once (bf16), H and d written once (fp32)."""
+    n, N = spec.d_in, spec.n_tok
+    return 2 * 2 * N * n + 2 * 4 * n * n
+
+
+def recorded_traffic(workload):
+    """(bytes per launch, description) of the dominant kernel on `workload`,
+    or (None, reason) when there is no record or the kernel changed since."""
+    import hashlib
+    try:
+        with open(TRAFFIC_RECORD) as f:
+            rec = json.load(f)
+        with open(KERNEL_SOURCE, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, ValueError):
+        return None, "no traffic record"
+    if rec.get("workload") != workload:
+        return None, f"traffic recorded for {rec.get('workload')}, not {workload}"
+    if rec.get("kernel_source_sha256") != sha:
+        return None, "kernel source changed since the traffic was captured"
+    return int(rec["bytes_per_launch_full_size"]), rec.get("how", "")
 
 
 # ----------------------------------------------------------------------------- oracle timing
@@ -470,6 +496,11 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": world * k2 / (ms_e2e / 1e3), "unit": UNIT, "steps": k2,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
+    # ---- the 224 layers of a 7B-shaped model, each on its own inputs
+    model = None
+    if not args.no_model_pass:
+        model = model_pass(args, rank, world, stream, barrier, max_over_ranks)
+
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -494,39 +525,64 @@ def run_ours(args, rank, world, local_rank):
             entry["bound"] = bound
         phase_out[name] = entry
 
-    # Dominant kernel: the persistent tcgen05 GEMM (kernel atb_bf16_kernel),
-    # launched once for the Hessian SYRK and once for the QEP cross product;
-    # each of those phases holds exactly that one launch.  Algorithmic flops
-    # per launch = (n(n+1)N + 2n^2 N) / 2, over the mean of the two launches'
-    # CUDA-event durations.  The bf16 peak is the sustained one: the kernel
-    # runs inside a long, power-capped step.
+    # Dominant kernel: the persistent tcgen05 product atb16_kernel, launched
+    # once for the Hessian (bf16) and once per token slice of the QEP cross
+    # product (fp16 operands; B200's dense fp16 and bf16 rates are the same).
+    # Its phases hold those launches plus a few small ones (the first slice's
+    # operand pass, column scales, two no-op fallback launches), so
+    # achieved = the phases' algorithmic flops over the phases' CUDA-event
+    # time, a lower bound on the kernel's own rate.  Peak: the measured bf16
+    # burst figure (the timed region is a fraction of a second); the
+    # sustained one is given beside it.
     gemm_phases = [p for p in ("hessian_syrk", "qep_cross") if p in phase_out]
     gemm_ms = sum(phase_out[p]["ms_per_step"] for p in gemm_phases)
-    gemm_launches = sum(phase_out[p]["launches_per_step"] for p in gemm_phases)
     gemm_flop = sum(work[p][0] for p in gemm_phases)
-    ms_launch = gemm_ms / gemm_launches
-    per_launch = gemm_flop / gemm_launches
-    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    achieved = per_launch / (ms_launch / 1e3) / 1e12
-    roof = {"bound": "tensor", "unit": "TFLOP/s", "kernel": "atb_bf16_kernel",
-            "phases": gemm_phases, "peak_source": f"{peak_src} bf16 sustained (of {peak_src})",
-            "achieved": round(achieved, 2), "peak": round(peak, 2),
-            "frac": round(achieved / peak, 4),
-            "traffic": None if args.n_tok else TRAFFIC_PER_LAUNCH.get(spec.name),
-            "per_launch": {"amount": per_launch, "unit": "flop", "ms": round(ms_launch, 4)}}
+    n_launch = 1 + (cross_slices(spec) if "qep_cross" in gemm_phases else 0)
+    per_launch = gemm_flop / n_launch
+    ms_launch = gemm_ms / n_launch
+    peak_b = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak_s = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    achieved = gemm_flop / (gemm_ms / 1e3) / 1e12
+    traffic, traffic_how = recorded_traffic(spec.name) if not args.n_tok else (None, "reduced token count")
     sm_mhz = clocks.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+    roof = {"bound": "tensor", "unit": "TFLOP/s", "kernel": "atb16_kernel", "phases": gemm_phases,
+            "achieved": round(achieved, 2), "peak": round(peak_b, 2),
+            "peak_source": f"bf16_tflops (burst) of {peak_src}", "frac": round(achieved / peak_b, 4),
+            "frac_of_sustained_peak": round(achieved / peak_s, 4), "sm_mhz_median": sm_mhz,
+            "traffic": traffic, "traffic_source": traffic_how,
+            "per_launch": {"launches": n_launch, "flop": per_launch, "ms": round(ms_launch, 4),
+                           "algorithmic_bytes": gemm_bytes(spec) / n_launch}}
 
-    # whole-layer roofline time: tensor phases at the bf16 peak, f32 phases at the
-    # fp32 peak of the tensor cores' 3xTF32 path is not used here: each phase at
-    # the peak of the unit it runs on today
+    # Whole-layer roofline: every phase at the peak of the unit it needs,
+    # taken in sequence: the bf16 products at the measured bf16 burst peak, the
+    # fp32-accurate products (3xTF32 on the tensor cores) at tf32's dense
+    # peak, taken as half the measured bf16 figure (the B200's nominal ratio,
+    # 1.1 vs 2.25 PFLOP/s), counting each product once, and the memory-bound
+    # phases at the measured copy bandwidth.
+    peak_tf32 = peak_b / 2.0
     t_roof = 0.0
     for name, (amt, unit, bound) in work.items():
+        if name == "hadamard_rotate" and not args.rotate:
+            continue
         if bound == "tensor":
-            t_roof += amt / (peaks.get("bf16_tflops_sustained", 1400.0) * 1e12)
+            t_roof += amt / (peak_b * 1e12)
         elif bound == "f32":
-            t_roof += amt / (f32_simt_peak_tflops(sm_mhz) * 1e12)
+            t_roof += amt / (peak_tf32 * 1e12)
         else:
-            t_roof += amt / (peaks.get("hbm_gbs", 6650.0) * 1e9)
+            t_roof += amt / (peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]) * 1e9)
+    layer_roof = {"t_roof_ms": round(t_roof * 1e3, 3), "t_measured_ms": round(ms_per_step, 3),
+                  "frac": round(t_roof * 1e3 / ms_per_step, 4),
+                  "peaks": {"bf16_tflops": peak_b, "tf32_tflops": peak_tf32, "tf32_from": "half the measured bf16 burst",
+                            "hbm_gbs": peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), "source": peak_src}}
+    for name, entry in phase_out.items():
+        amt, unit, bound = work.get(name, (0, "", ""))
+        if "achieved_tflops" in entry:
+            pk = peak_b if bound == "tensor" else peak_tf32
+            entry["frac_of_peak"] = round(entry["achieved_tflops"] / pk, 4)
+            if bound == "f32":
+                entry["tensor_issue_frac"] = round(3 * entry["achieved_tflops"] / pk, 4)
+        elif "achieved_gbs" in entry:
+            entry["frac_of_peak"] = round(entry["achieved_gbs"] / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), 4)
 
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
@@ -536,10 +592,11 @@ def run_ours(args, rank, world, local_rank):
         "config": dict(workload_config(spec),
                        parallelism=(f"{world} independent layers, one per rank" if world > 1
                                     else "single GPU")),
+        "seconds_per_7b_model": model["seconds"] if model else None,
+        "model_pass": model,
         "seconds_per_224_layers_of_this_shape": round(224 * ms_per_step / 1e3, 3),
         "three_calls_ms_per_step": round(ms_three, 3),
-        "layer_roofline_ms_current_units": round(t_roof * 1e3, 3),
-        "roofline": roof, "phases": phase_out, "gpu_launches": int(launches),
+        "roofline": roof, "layer_roofline": layer_roof, "phases": phase_out, "gpu_launches": int(launches),
         "clocks": clocks, "e2e": e2e,
     }
     if args.rotate:
@@ -552,6 +609,57 @@ def run_ours(args, rank, world, local_rank):
                                 "sample": cpu_sample_text(spec),
                                 "cpu_seconds_measured": round(t_meas, 2)}
     print(json.dumps(line), flush=True)
+
+
+def model_pass(args, rank, world, stream, barrier, max_over_ranks):
+    """All 224 linear layers of a 32-block Llama-2-7B-shaped model, each with its
+    own seeded synthetic calibration inputs (131072 tokens, Student-t(4) with 1%
+    of channels x20, Xhat = X + 2% channel noise) and weight (bf16 N(0, 0.02^2)),
+    attention layers at 4 bits and MLP layers at 3 bits, g128, QEP alpha 0.5,
+    damp 0.01, act_order off: one oc_quantize_layer call per layer.  Inputs are
+    drawn on the device before each layer, outside its CUDA events; the
+    reported seconds are the sum of the layers' device times (max over ranks;
+    rank r takes layers r, r + N, ...)."""
+    import torch
+
+    import post_weight_quantization_07_b200 as oc
+    from synthetic import llama7b_layers, make_layer_device
+
+    specs = llama7b_layers(args.model_tokens)
+    total_ms = 0.0
+    done = 0
+    launches0 = oc.oc_launch_count()
+    t_wall = time.perf_counter()
+    for i, spec in enumerate(specs):
+        if i % world != rank:
+            continue
+        L = make_layer_device(spec, "cuda")
+        m, n, G = spec.d_out, spec.d_in, spec.groupsize
+        outs = dict(H=torch.empty(n, n, device="cuda"), W_out=torch.empty_like(L["W"]),
+                    codes=torch.empty(m, n * spec.wbits // 32, dtype=torch.int32, device="cuda"),
+                    scales=torch.empty(m, n // G, device="cuda"), zeros=torch.empty(m, n // G, device="cuda"))
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        oc.oc_quantize_layer(L["W"], L["X"], L["Xhat"], spec.alpha, spec.damp, spec.wbits, spec.groupsize,
+                             spec.act_order, stream=stream, **outs)
+        b.record(stream)
+        b.synchronize()
+        total_ms += a.elapsed_time(b)
+        done += 1
+        del L, outs
+    st = oc.oc_stream_status(stream)
+    if st != oc.OC_OK:
+        raise RuntimeError(f"model pass failed: {oc.oc_status_string(st)}")
+    barrier()
+    ms = max_over_ranks(total_ms)
+    return {"seconds": round(ms / 1e3, 3), "layers": len(specs), "layers_per_rank": done,
+            "layers_per_s": round(len(specs) / (ms / 1e3), 3), "calibration_tokens": args.model_tokens,
+            "gpu_launches": int(oc.oc_launch_count() - launches0),
+            "wall_s_including_input_generation": round(time.perf_counter() - t_wall, 1),
+            "what": ("224 layers (32 blocks x q/k/v/o 4096x4096 4-bit, gate/up 4096->11008 and down "
+                     "11008->4096 3-bit, g128), each on its own seeded inputs, one oc_quantize_layer call "
+                     "per layer; sum of the layers' device times, input generation excluded")}
 
 
 # ----------------------------------------------------------------------------- one layer over N GPUs
@@ -922,6 +1030,10 @@ def main():
                     help="calibration tokens per layer (default: the workload's own)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-model-pass", action="store_true",
+                    help="skip the 224-layer 7B-shaped model pass (seconds per model)")
+    ap.add_argument("--model-tokens", type=int, default=131072,
+                    help="calibration tokens per layer in the model pass")
     ap.add_argument("--rotate", type=int, default=0, metavar="B",
                     help="rotate W, X, Xhat by a block-B Hadamard matrix every step before quantising")
     ap.add_argument("--gemv-batch", type=int, default=1,

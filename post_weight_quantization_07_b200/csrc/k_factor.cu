@@ -609,4 +609,98 @@ void factor_inverse_upper(const Ctx& c, float* M, float* X, float* scratch, floa
   check_cuda(cudaGraphLaunch(exec, c.stream), "cudaGraphLaunch(factor)");
 }
 
+namespace {
+
+// Sets the graph's condition: 1 when GPTQ's preparation found dead columns.
+__global__ void set_dead_condition_kernel(cudaGraphConditionalHandle h, const DiagStats* stats) {
+  cudaGraphSetConditional(h, stats->n_dead > 0 ? 1u : 0u);
+}
+
+struct SelectGraph {
+  int device;
+  int64_t n;
+  const void *H, *perm, *stats_g, *stats_q, *Ug, *Uq, *X, *scratch, *split, *status;
+  cudaGraphExec_t exec;
+};
+std::vector<SelectGraph> g_select_graphs;
+
+}  // namespace
+
+void qep_factor_select(const Ctx& c, const float* H, int64_t n, const int32_t* perm, const DiagStats* stats_g,
+                       const DiagStats* stats_q, const float* Ug, float* Uq, float* X, float* scratch, float* split) {
+  for (const SelectGraph& g : g_select_graphs) {
+    if (g.device == c.device && g.n == n && g.H == H && g.perm == perm && g.stats_g == stats_g &&
+        g.stats_q == stats_q && g.Ug == Ug && g.Uq == Uq && g.X == X && g.scratch == scratch && g.split == split &&
+        g.status == c.status) {
+      check_cuda(cudaGraphLaunch(g.exec, c.stream), "cudaGraphLaunch(select)");
+      count_launches(1);
+      return;
+    }
+  }
+  // One graph: a kernel that reads the dead-column count on the device, then
+  // an if/else node.  If: QEP's own matrix H + lam I (no dead-column fix, lam
+  // from stats_q) in processing order, factored into Uq.  Else: Uq = Ug.
+  cudaGraph_t graph = nullptr;
+  check_cuda(cudaGraphCreate(&graph, 0), "cudaGraphCreate(select)");
+  cudaGraphExec_t exec = nullptr;
+  static cudaStream_t capture_stream[64] = {};
+  try {
+    cudaGraphConditionalHandle h;
+    check_cuda(cudaGraphConditionalHandleCreate(&h, graph, 0, cudaGraphCondAssignDefault),
+               "cudaGraphConditionalHandleCreate");
+    cudaKernelNodeParams kp = {};
+    void* args[2] = {&h, const_cast<DiagStats**>(&stats_g)};
+    kp.func = reinterpret_cast<void*>(set_dead_condition_kernel);
+    kp.gridDim = dim3(1);
+    kp.blockDim = dim3(1);
+    kp.kernelParams = args;
+    cudaGraphNode_t setter = nullptr;
+    check_cuda(cudaGraphAddKernelNode(&setter, graph, nullptr, 0, &kp), "cudaGraphAddKernelNode(select)");
+    cudaGraphNodeParams cp = {};
+    cp.type = cudaGraphNodeTypeConditional;
+    cp.conditional.handle = h;
+    cp.conditional.type = cudaGraphCondTypeIf;
+    cp.conditional.size = 2;
+    cudaGraphNode_t cond = nullptr;
+    check_cuda(cudaGraphAddNode(&cond, graph, &setter, 1, &cp), "cudaGraphAddNode(conditional)");
+    cudaGraph_t body_dead = cp.conditional.phGraph_out[0];
+    cudaGraph_t body_live = cp.conditional.phGraph_out[1];
+    if (capture_stream[c.device & 63] == nullptr)
+      check_cuda(cudaStreamCreateWithFlags(&capture_stream[c.device & 63], cudaStreamNonBlocking),
+                 "cudaStreamCreate(capture)");
+    Ctx cc = c;
+    cc.stream = capture_stream[c.device & 63];
+    check_cuda(cudaStreamBeginCaptureToGraph(cc.stream, body_dead, nullptr, nullptr, 0,
+                                             cudaStreamCaptureModeThreadLocal),
+               "cudaStreamBeginCaptureToGraph(dead)");
+    try {
+      launch_build_reversed(cc, H, n, perm, stats_q, 1.0f, false, Uq);
+      factor_direct(cc, Uq, X, scratch, Uq, n, split);
+    } catch (...) {
+      cudaStreamEndCapture(cc.stream, &body_dead);
+      throw;
+    }
+    check_cuda(cudaStreamEndCapture(cc.stream, &body_dead), "cudaStreamEndCapture(dead)");
+    check_cuda(cudaStreamBeginCaptureToGraph(cc.stream, body_live, nullptr, nullptr, 0,
+                                             cudaStreamCaptureModeThreadLocal),
+               "cudaStreamBeginCaptureToGraph(live)");
+    const cudaError_t e = cudaMemcpyAsync(Uq, Ug, static_cast<size_t>(n) * n * sizeof(float),
+                                          cudaMemcpyDeviceToDevice, cc.stream);
+    check_cuda(cudaStreamEndCapture(cc.stream, &body_live), "cudaStreamEndCapture(live)");
+    check_cuda(e, "copy factor");
+    check_cuda(cudaGraphInstantiate(&exec, graph, 0), "cudaGraphInstantiate(select)");
+  } catch (...) {
+    cudaGraphDestroy(graph);
+    throw;
+  }
+  cudaGraphDestroy(graph);
+  if (g_select_graphs.size() >= 8) {
+    cudaGraphExecDestroy(g_select_graphs.front().exec);
+    g_select_graphs.erase(g_select_graphs.begin());
+  }
+  g_select_graphs.push_back({c.device, n, H, perm, stats_g, stats_q, Ug, Uq, X, scratch, split, c.status, exec});
+  check_cuda(cudaGraphLaunch(exec, c.stream), "cudaGraphLaunch(select)");
+  count_launches(1);
+}
+
 }  // namespace oc

@@ -55,6 +55,11 @@ struct Params {
   float alpha;
   int accumulate;
   int* status;
+  // optional device flags, zero when the operand's lo half is all zero (the
+  // operand is exact in tf32, e.g. bf16-valued weights): its correction MMA
+  // adds nothing and is skipped
+  const int* a_lo_nz;
+  const int* b_lo_nz;
 };
 
 // Tiles wholly above the diagonal are skipped when only the lower triangle of
@@ -170,6 +175,8 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constan
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc = instr_desc(2, 2, false, false, BM, BN);
+    const bool use_al = p.a_lo_nz == nullptr || *p.a_lo_nz != 0;
+    const bool use_bl = p.b_lo_nz == nullptr || *p.b_lo_nz != 0;
     uint64_t consumed = 0;
     int it = 0;
     bool ok = true;
@@ -205,10 +212,10 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_constan
               const uint64_t al = smem_desc_sw128(sal + kk * 32, 16, 1024);
               const uint64_t bh = smem_desc_sw128(sbh + kk * 32, 16, 1024);
               const uint64_t bl = smem_desc_sw128(sbl + kk * 32, 16, 1024);
-              const uint32_t first = (k0 == s0 && kk == 0) ? 0u : 1u;
-              mma_tf32_ss(dcol, al, bh, idesc, first);
-              mma_tf32_ss(dcol, ah, bl, idesc, 1u);
-              mma_tf32_ss(dcol, ah, bh, idesc, 1u);
+              uint32_t accf = (k0 == s0 && kk == 0) ? 0u : 1u;
+              if (use_al) { mma_tf32_ss(dcol, al, bh, idesc, accf); accf = 1u; }
+              if (use_bl) { mma_tf32_ss(dcol, ah, bl, idesc, accf); accf = 1u; }
+              mma_tf32_ss(dcol, ah, bh, idesc, accf);
             }
             mma_commit(&empty[s]);
           }
@@ -452,6 +459,8 @@ gemm_tf32x3_pair_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_co
     if (leader) {
       // ---------------------------------------------------------------- MMA issuer (leader)
       constexpr uint32_t idesc = instr_desc(2, 2, false, false, PM, PN);
+      const bool use_al = p.a_lo_nz == nullptr || *p.a_lo_nz != 0;
+      const bool use_bl = p.b_lo_nz == nullptr || *p.b_lo_nz != 0;
       uint64_t consumed = 0;
       int it = 0;
       bool ok = true;
@@ -487,10 +496,10 @@ gemm_tf32x3_pair_kernel(const __grid_constant__ CUtensorMap mAh, const __grid_co
                 const uint64_t al = smem_desc_sw128(sal + kk * 32, 16, 1024);
                 const uint64_t bh = smem_desc_sw128(sbh + kk * 32, 16, 1024);
                 const uint64_t bl = smem_desc_sw128(sbl + kk * 32, 16, 1024);
-                const uint32_t first = (k0 == s0 && kk == 0) ? 0u : 1u;
-                mma_tf32_ss_pair(dcol, al, bh, idesc, first);
-                mma_tf32_ss_pair(dcol, ah, bl, idesc, 1u);
-                mma_tf32_ss_pair(dcol, ah, bh, idesc, 1u);
+                uint32_t accf = (k0 == s0 && kk == 0) ? 0u : 1u;
+                if (use_al) { mma_tf32_ss_pair(dcol, al, bh, idesc, accf); accf = 1u; }
+                if (use_bl) { mma_tf32_ss_pair(dcol, ah, bl, idesc, accf); accf = 1u; }
+                mma_tf32_ss_pair(dcol, ah, bh, idesc, accf);
               }
               mma_commit_pair(&empty[s], kPairMask);
             }
@@ -651,9 +660,10 @@ __device__ __forceinline__ void split4(const float4 x, float4& h, float4& l) {
 
 __global__ void __launch_bounds__(256) split_tf32_v4_kernel(const float4* __restrict__ src, int64_t rows,
                                                             int64_t cols4, int64_t lds4, float4* __restrict__ hi,
-                                                            float4* __restrict__ lo, int64_t ldd4) {
+                                                            float4* __restrict__ lo, int64_t ldd4, int* lo_nz) {
   const int64_t total = rows * cols4;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  bool nz = false;
   for (int64_t e0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e0 < total; e0 += 4 * stride) {
     float4 x[4];
 #pragma unroll
@@ -670,9 +680,11 @@ __global__ void __launch_bounds__(256) split_tf32_v4_kernel(const float4* __rest
         const int64_t d = (e / cols4) * ldd4 + e % cols4;
         hi[d] = h;
         lo[d] = l;
+        nz |= (l.x != 0.f) | (l.y != 0.f) | (l.z != 0.f) | (l.w != 0.f);
       }
     }
   }
+  if (lo_nz != nullptr && nz) *lo_nz = 1;
 }
 
 // Vectorised transposing split through 64 x 64 tiles (rows and cols multiples
@@ -724,8 +736,13 @@ void set_attr_once(int device) {
 }  // namespace
 
 void split_tf32(const Ctx& c, const float* src, int64_t rows, int64_t cols, int64_t lds, float* hi, float* lo,
-                int64_t ldd, bool transpose) {
+                int64_t ldd, bool transpose, int* lo_nz) {
   if (rows <= 0 || cols <= 0) return;
+  if (lo_nz != nullptr) {
+    if (transpose || !(aligned16(src) && aligned16(hi) && aligned16(lo) && lds % 4 == 0 && ldd % 4 == 0 && cols % 4 == 0))
+      fail(OC_ERR_INVALID_ARG, "split_tf32: the lo flag needs the vectorised untransposed split");
+    check_cuda(cudaMemsetAsync(lo_nz, 0, sizeof(int), c.stream), "clear lo flag");
+  }
   const bool vec = aligned16(src) && aligned16(hi) && aligned16(lo) && lds % 4 == 0 && ldd % 4 == 0 &&
                    cols % 4 == 0 && (!transpose || rows % 4 == 0);
   if (vec && transpose && (rows + TT - 1) / TT <= 65535) {
@@ -739,7 +756,7 @@ void split_tf32(const Ctx& c, const float* src, int64_t rows, int64_t cols, int6
     const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(c.sm_count) * 8));
     split_tf32_v4_kernel<<<grid, 256, 0, c.stream>>>(reinterpret_cast<const float4*>(src), rows, cols / 4, lds / 4,
                                                      reinterpret_cast<float4*>(hi), reinterpret_cast<float4*>(lo),
-                                                     ldd / 4);
+                                                     ldd / 4, lo_nz);
     check_launch("split_tf32_v4_kernel");
     return;
   }
@@ -758,7 +775,7 @@ void split_tf32(const Ctx& c, const float* src, int64_t rows, int64_t cols, int6
 
 void gemm_tf32x3(const Ctx& c, int64_t M, int64_t N, int64_t K, float alpha, const float* A_hi,
                  const float* A_lo, int64_t lda, const float* B_hi, const float* B_lo, int64_t ldb,
-                 bool accumulate, float* C, int64_t ldc, unsigned flags) {
+                 bool accumulate, float* C, int64_t ldc, unsigned flags, const int* a_lo_nz, const int* b_lo_nz) {
   if (M <= 0 || N <= 0) return;
   if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || K > (int64_t(1) << 30))
     fail(OC_ERR_INVALID_ARG, "gemm_tf32x3: size too large");
@@ -777,6 +794,8 @@ void gemm_tf32x3(const Ctx& c, int64_t M, int64_t N, int64_t K, float alpha, con
   p.alpha = alpha;
   p.accumulate = accumulate ? 1 : 0;
   p.status = c.status;
+  p.a_lo_nz = a_lo_nz;
+  p.b_lo_nz = b_lo_nz;
   // A product with at least a wave of 256 x 256 tiles runs on CTA pairs (half
   // the operand traffic per SM); smaller ones keep more, smaller tiles.
   const int64_t pair_tiles = ((M + PM - 1) / PM) * ((N + PN - 1) / PN);

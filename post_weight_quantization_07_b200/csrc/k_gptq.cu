@@ -28,7 +28,8 @@ __device__ __forceinline__ void grid_from_minmax(float xmin, float xmax, float m
   z = fminf(fmaxf(rintf(-xmin / s), 0.f), maxq);
 }
 
-// Wp[r][j] = dead[p(j)] ? 0 : W[r][p(j)], one block per row (row staged in shared memory).
+// Wp[r][j] = dead[p(j)] ? 0 : W[r][p(j)] (dead may be null: no zeroing), one
+// block per row (row staged in shared memory).
 __global__ void permute_w_kernel(const float* __restrict__ W, int64_t n, const int32_t* __restrict__ perm,
                                  const unsigned char* __restrict__ dead, float* __restrict__ Wp) {
   extern __shared__ float row[];
@@ -37,7 +38,7 @@ __global__ void permute_w_kernel(const float* __restrict__ W, int64_t n, const i
   __syncthreads();
   for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
     const int64_t p = perm[j];
-    Wp[r * n + j] = dead[p] ? 0.f : row[p];
+    Wp[r * n + j] = (dead != nullptr && dead[p]) ? 0.f : row[p];
   }
 }
 
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(SweepShape<LPR>::THREADS, 2)
 sweep_block_kernel(float* __restrict__ Wp, int64_t m, int64_t n, const float* __restrict__ U, int64_t j1, int G,
                    float maxq, int static_groups, const int32_t* __restrict__ perm, float* __restrict__ scales,
                    float* __restrict__ zeros, unsigned char* __restrict__ codes8, float* __restrict__ Err,
-                   float* __restrict__ Err_lo) {
+                   float* __restrict__ Err_lo, int64_t err_ld) {
   using S = SweepShape<LPR>;
   constexpr int CPL = S::CPL;
   constexpr int NT = S::THREADS;
@@ -292,13 +293,13 @@ sweep_block_kernel(float* __restrict__ Wp, int64_t m, int64_t n, const float* __
             h[k] = tf32_rna(ev[i + k]);
             l[k] = tf32_rna(ev[i + k] - h[k]);
           }
-          *reinterpret_cast<float4*>(Err + r * SB + CPL * q + i) = make_float4(h[0], h[1], h[2], h[3]);
-          *reinterpret_cast<float4*>(Err_lo + r * SB + CPL * q + i) = make_float4(l[0], l[1], l[2], l[3]);
+          *reinterpret_cast<float4*>(Err + r * err_ld + CPL * q + i) = make_float4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<float4*>(Err_lo + r * err_ld + CPL * q + i) = make_float4(l[0], l[1], l[2], l[3]);
         }
       } else {
 #pragma unroll
         for (int i = 0; i < CPL; i += 4)
-          *reinterpret_cast<float4*>(Err + r * SB + CPL * q + i) = make_float4(ev[i], ev[i + 1], ev[i + 2], ev[i + 3]);
+          *reinterpret_cast<float4*>(Err + r * err_ld + CPL * q + i) = make_float4(ev[i], ev[i + 1], ev[i + 2], ev[i + 3]);
       }
     }
   }
@@ -379,7 +380,7 @@ constexpr int kSweepLPR = 32;
 template <int LPR, bool SMALLG>
 void launch_sweep_shape(const Ctx& c, float* Wp, int64_t m, int64_t n, const float* U, int64_t j1, int G,
                         float maxq, bool static_groups, const int32_t* perm, float* scales, float* zeros,
-                        unsigned char* codes8, float* Err, float* Err_lo) {
+                        unsigned char* codes8, float* Err, float* Err_lo, int64_t err_ld) {
   using S = SweepShape<LPR>;
   static bool attr_done[64] = {false};
   if (!attr_done[c.device & 63]) {
@@ -391,7 +392,7 @@ void launch_sweep_shape(const Ctx& c, float* Wp, int64_t m, int64_t n, const flo
   const int64_t want = (m + SWEEP_ROWS - 1) / SWEEP_ROWS;
   const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(c.sm_count) * 2));
   sweep_block_kernel<LPR, SMALLG><<<grid, S::THREADS, S::SMEM, c.stream>>>(
-      Wp, m, n, U, j1, G, maxq, static_groups ? 1 : 0, perm, scales, zeros, codes8, Err, Err_lo);
+      Wp, m, n, U, j1, G, maxq, static_groups ? 1 : 0, perm, scales, zeros, codes8, Err, Err_lo, err_ld);
   check_launch("sweep_block_kernel");
 }
 
@@ -399,15 +400,16 @@ void launch_sweep_shape(const Ctx& c, float* Wp, int64_t m, int64_t n, const flo
 
 void launch_sweep_block(const Ctx& c, float* Wp, int64_t m, int64_t n, const float* U, int64_t j1, int G,
                         int wbits, bool static_groups, const int32_t* perm, float* scales, float* zeros,
-                        unsigned char* codes8, float* Err, float* Err_lo) {
+                        unsigned char* codes8, float* Err, float* Err_lo, int64_t err_ld) {
   constexpr int LPR = kSweepLPR;
   const float maxq = static_cast<float>((1 << wbits) - 1);
+  if (err_ld < SB || err_ld % 4) fail(OC_ERR_INVALID_ARG, "sweep: error leading dimension");
   if (!static_groups && G < SB / LPR)
     launch_sweep_shape<LPR, true>(c, Wp, m, n, U, j1, G, maxq, static_groups, perm, scales, zeros, codes8, Err,
-                                  Err_lo);
+                                  Err_lo, err_ld);
   else
     launch_sweep_shape<LPR, false>(c, Wp, m, n, U, j1, G, maxq, static_groups, perm, scales, zeros, codes8, Err,
-                                   Err_lo);
+                                   Err_lo, err_ld);
 }
 
 void launch_pack(const Ctx& c, const unsigned char* codes8, int64_t m, int64_t n, int wbits,

@@ -216,24 +216,41 @@ void check_gptq_args(const float* W, int64_t m, int64_t n, int wbits, int groups
 
 // GPTQ after the factor: blocked sweep over the permuted working copy Wp with
 // tensor-core trailing updates, then packing (and the processing order out).
+// Lazy updates on two levels: the errors of each 128-column block update the
+// rest of its 512-column superblock at once (k = 128); at the end of a
+// superblock, its 512 columns of errors update every later column in one
+// product (k = 512), so the wide updates pass over W a quarter as often.
+// Errh, Errl: m x kSuperBlock each.
 void gptq_sweep_and_pack(const Ctx& c, float* Wp, int64_t m, int64_t n, const float* U, const float* UTh,
                          const float* UTl, int G, int wbits, bool act_order, int32_t* perm, float* scales,
                          float* zeros, unsigned char* codes8, float* Errh, float* Errl, uint32_t* codes,
                          int32_t* perm_out) {
-  for (int64_t j1 = 0; j1 < n; j1 += 128) {
-    const int64_t bw = std::min<int64_t>(128, n - j1);
-    const int64_t j2 = j1 + bw;
-    {
-      // the sweep writes the block's errors already split for 3xTF32
-      PhaseScope ps(c, kPhGptqSweep);
-      launch_sweep_block(c, Wp, m, n, U, j1, G, wbits, act_order, perm, scales, zeros, codes8, Errh, Errl);
+  constexpr int64_t SBW = kSuperBlock;
+  for (int64_t s1 = 0; s1 < n; s1 += SBW) {
+    const int64_t s2 = std::min(n, s1 + SBW);
+    for (int64_t j1 = s1; j1 < s2; j1 += 128) {
+      const int64_t bw = std::min<int64_t>(128, s2 - j1);
+      const int64_t j2 = j1 + bw;
+      float* eh = Errh + (j1 - s1);
+      float* el = Errl + (j1 - s1);
+      {
+        // the sweep writes the block's errors already split for 3xTF32
+        PhaseScope ps(c, kPhGptqSweep);
+        launch_sweep_block(c, Wp, m, n, U, j1, G, wbits, act_order, perm, scales, zeros, codes8, eh, el, SBW);
+      }
+      if (j2 < s2) {
+        // W[:, j2:s2] -= Err U[j1:j2, j2:s2] on the tensor cores (3xTF32); B
+        // stored = U^T[j2:s2, j1:j2] (rows j2.., columns j1..j2 of the transpose)
+        PhaseScope ps(c, kPhGptqTrailing);
+        gemm_tf32x3(c, m, s2 - j2, bw, -1.f, eh, el, SBW, UTh + j2 * n + j1, UTl + j2 * n + j1, n, true, Wp + j2,
+                    n, kANone);
+      }
     }
-    if (j2 < n) {
-      // W[:, j2:] -= Err U[j1:j2, j2:] on the tensor cores (3xTF32); B stored
-      // = U^T[j2:, j1:j2] (rows j2.., columns j1..j1+bw of the transpose)
+    if (s2 < n) {
+      // W[:, s2:] -= ErrS U[s1:s2, s2:] (k = s2 - s1)
       PhaseScope ps(c, kPhGptqTrailing);
-      gemm_tf32x3(c, m, n - j2, bw, -1.f, Errh, Errl, 128, UTh + j2 * n + j1, UTl + j2 * n + j1, n, true, Wp + j2,
-                  n, kANone);
+      gemm_tf32x3(c, m, n - s2, s2 - s1, -1.f, Errh, Errl, SBW, UTh + s2 * n + s1, UTl + s2 * n + s1, n, true,
+                  Wp + s2, n, kANone);
     }
   }
   {
@@ -293,11 +310,12 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
   sizing.take<float>(mn * count);         // G -> T, one per layer
   sizing.take<float>(mn);                 // permuted working copy of W
   sizing.take<unsigned char>(mn);         // codes, processing order
-  sizing.take<float>(2 * static_cast<size_t>(m_max) * 128);  // block errors, hi and lo halves
+  sizing.take<float>(2 * static_cast<size_t>(m_max) * kSuperBlock);  // superblock errors, hi and lo halves
   sizing.take<int32_t>(2 * static_cast<size_t>(n));          // order | inverse
   sizing.take<unsigned char>(n);          // dead-column mask
   sizing.take<float>(factor_split_floats(n));
-  sizing.take<DiagStats>(1);
+  sizing.take<DiagStats>(2);              // GPTQ's and QEP's dampening
+  sizing.take<int>(1);                    // W's tf32 lo-half flag
   const size_t cross_bytes = terms_given ? 0 : cross_scratch_bytes(n_tok, n);
   sizing.take<unsigned char>(cross_bytes);  // the cross product's operands
   Carve cv{workspace(c, sizing.off + 256)};
@@ -312,12 +330,14 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
   float* Gs = cv.take<float>(mn * count);
   float* Wp = cv.take<float>(mn);
   unsigned char* codes8 = cv.take<unsigned char>(mn);
-  float* Errh = cv.take<float>(2 * static_cast<size_t>(m_max) * 128);
-  float* Errl = Errh + static_cast<size_t>(m_max) * 128;
+  float* Errh = cv.take<float>(2 * static_cast<size_t>(m_max) * kSuperBlock);
+  float* Errl = Errh + static_cast<size_t>(m_max) * kSuperBlock;
   int32_t* perm = cv.take<int32_t>(2 * static_cast<size_t>(n));
   unsigned char* dead = cv.take<unsigned char>(n);
   float* fsplit = cv.take<float>(factor_split_floats(n));
-  DiagStats* stats = cv.take<DiagStats>(1);
+  DiagStats* stats = cv.take<DiagStats>(2);
+  DiagStats* stats_q = stats + 1;
+  int* lo_flag = cv.take<int>(1);
   unsigned char* cross_scratch = cv.take<unsigned char>(cross_bytes);
   auto Gl = [&](int l) { return Gs + static_cast<size_t>(l) * mn; };
   const size_t nn_bytes = nn * sizeof(float);
@@ -336,125 +356,92 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
       launch_mirror_upper(c, H, n);
     }
   }
-  // GPTQ's dampened Hessian equals QEP's 2A unless a column is dead (their
-  // dampening constants then differ): one device-to-host read decides.
+  // GPTQ's preparation: dead-column mask and dampening constant (device only;
+  // a non-finite diagonal is recorded in the status word and the call runs
+  // to its end on the bad values).
   launch_diag_stats(c, H, n, damp, 1.0f, true, stats, dead);
-  DiagStats hs{};
-  check_cuda(cudaMemcpyAsync(&hs, stats, sizeof(DiagStats), cudaMemcpyDeviceToHost, c.stream), "read stats");
-  check_cuda(cudaStreamSynchronize(c.stream), "cudaStreamSynchronize");
-  if (hs.nonfinite) return finish(c);
-  // The factorisation needs only H.  With no dead column (one factorisation
-  // serves QEP and GPTQ) it runs on a side stream, on a few SMs, while the
-  // cross product X^T Xhat occupies the rest; it factors into UTh (input
-  // reversed and dampened, output U) with UTl and Fs as its scratch.
-  const bool shared_factor = hs.n_dead == 0;
+  // GPTQ's inverse factor needs only H: it runs on a side stream, on a few
+  // SMs, while the cross product X^T Xhat occupies the rest; it factors into
+  // UTh (input reversed and dampened, output U) with UTl, Fs and fsplit as
+  // its scratch.
   SideStream& ss = side_stream(c.device);
   Ctx cs = c;
   cs.stream = ss.stream;
-  if (shared_factor) {
-    check_cuda(cudaEventRecord(ss.fork, c.stream), "cudaEventRecord(fork)");
-    check_cuda(cudaStreamWaitEvent(cs.stream, ss.fork, 0), "cudaStreamWaitEvent(fork)");
+  check_cuda(cudaEventRecord(ss.fork, c.stream), "cudaEventRecord(fork)");
+  check_cuda(cudaStreamWaitEvent(cs.stream, ss.fork, 0), "cudaStreamWaitEvent(fork)");
+  {
     PhaseScope ps(cs, kPhFactor);
     if (act_order) launch_act_order_perm(cs, H, n, perm);
     else launch_identity_perm(cs, n, perm);
     launch_build_reversed(cs, H, n, perm, stats, 1.0f, true, UTh);
     factor_inverse_upper(cs, UTh, UTl, Fs, UTh, n, true, fsplit);
-    check_cuda(cudaEventRecord(ss.join, cs.stream), "cudaEventRecord(join)");
   }
+  check_cuda(cudaEventRecord(ss.join, cs.stream), "cudaEventRecord(join)");
   if (terms_given) {
     check_cuda(cudaMemcpyAsync(D, D_in, nn_bytes, cudaMemcpyDeviceToDevice, c.stream), "copy d");
   } else {
-    {
-      // d = (X - Xhat)^T Xhat in token ranges: between two launches the
-      // high-priority factorisation can take the freed SMs for its wide
-      // tensor-core products
-      PhaseScope ps(c, kPhQepCross);
-      const int parts = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens)));
-      launch_cross_product(c, X, Xhat, n_tok, n, H, D, cross_scratch, parts,
-                           shared_factor ? c.sm_count - kSideSMs : 0);
-    }
+    // d = (X - Xhat)^T Xhat in token ranges: between two launches the
+    // high-priority factorisation can take the freed SMs for its wide
+    // tensor-core products
+    PhaseScope ps(c, kPhQepCross);
+    const int parts = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kCrossParts, n_tok / kCrossPartMinTokens)));
+    launch_cross_product(c, X, Xhat, n_tok, n, H, D, cross_scratch, parts, c.sm_count - kSideSMs);
   }
   {
     // G = W d for every layer while the split copies of d^T are live
     PhaseScope ps(c, kPhQepWDelta);
     split_tf32(c, D, n, n, n, Xi, scratch, n, true);
     for (int l = 0; l < count; ++l) {
-      split_tf32(c, W[l], m[l], n, n, Ph, Pl, n);
-      gemm_tf32x3(c, m[l], n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, Gl(l), n, kANone);
+      // bf16-valued weights are exact in tf32: W_lo = 0 skips a third of the MMAs
+      split_tf32(c, W[l], m[l], n, n, Ph, Pl, n, false, lo_flag);
+      gemm_tf32x3(c, m[l], n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, Gl(l), n, kANone, lo_flag);
     }
   }
-  if (!shared_factor) {
-    // two factorisations: QEP's own (original order), then GPTQ's
-    {
-      PhaseScope ps(c, kPhFactor);
-      DiagStats* qs = stats;
-      launch_diag_stats(c, H, n, damp, 1.0f, false, qs, nullptr);
-      launch_build_reversed(c, H, n, nullptr, qs, 1.0f, false, D);
-      factor_inverse_upper(c, D, Xi, scratch, D, n, true, fsplit);
-    }
-    {
-      PhaseScope ps(c, kPhQepApply);
-      split_tf32(c, D, n, n, n, Xi, scratch, n);
-      split_tf32(c, D, n, n, n, UTh, UTl, n, true);
-      for (int l = 0; l < count; ++l) {
-        const size_t ml = static_cast<size_t>(m[l]) * n;
-        split_tf32(c, Gl(l), m[l], n, n, Ph, Pl, n);
-        gemm_tf32x3(c, m[l], n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, Gl(l), n, kBLower);
-        split_tf32(c, Gl(l), m[l], n, n, Ph, Pl, n);
-        launch_copy_f32(c, W[l], W_out[l], static_cast<int64_t>(ml));
-        gemm_tf32x3(c, m[l], n, n, 2.f * alpha, Ph, Pl, n, UTh, UTl, n, true, W_out[l], n, kBUpper);
-      }
-    }
-    {
-      PhaseScope ps(c, kPhFactor);
-      launch_diag_stats(c, H, n, damp, 1.0f, true, stats, dead);
-      if (act_order) launch_act_order_perm(c, H, n, perm);
-      else launch_identity_perm(c, n, perm);
-      launch_build_reversed(c, H, n, perm, stats, 1.0f, true, D);
-      factor_inverse_upper(c, D, Xi, scratch, D, n, true, fsplit);
-    }
-    {
-      PhaseScope ps(c, kPhGptqPrep);
-      split_tf32(c, D, n, n, n, UTh, UTl, n, true);
-    }
-    for (int l = 0; l < count; ++l) {
-      {
-        PhaseScope ps(c, kPhGptqPrep);
-        launch_permute_w(c, W_out[l], m[l], n, perm, dead, Wp);
-        if (act_order) launch_static_grid(c, W_out[l], m[l], n, static_cast<int>(G), wbits, dead, scales[l], zeros[l]);
-      }
-      gptq_sweep_and_pack(c, Wp, m[l], n, D, UTh, UTl, static_cast<int>(G), wbits, act_order != 0, perm, scales[l],
-                          zeros[l], codes8, Errh, Errl, codes[l], l == 0 ? perm_out : nullptr);
-    }
-    return finish(c);
-  }
-
   check_cuda(cudaStreamWaitEvent(c.stream, ss.join, 0), "cudaStreamWaitEvent(join)");
   {
+    // QEP's factor Uq into D: GPTQ's when no column is dead (its dampened
+    // Hessian then equals QEP's 2A), else QEP's own in the same processing
+    // order (the two dampening constants differ): decided on the device.
+    PhaseScope ps(c, kPhFactor);
+    launch_diag_stats(c, H, n, damp, 1.0f, false, stats_q, nullptr);
+    qep_factor_select(c, H, n, perm, stats, stats_q, UTh, D, Xi, scratch, fsplit);
+  }
+  {
     PhaseScope ps(c, kPhQepApply);
-    check_cuda(cudaMemcpyAsync(D, UTh, nn_bytes, cudaMemcpyDeviceToDevice, c.stream), "copy U");
-    split_tf32(c, D, n, n, n, Xi, scratch, n);
-    split_tf32(c, D, n, n, n, UTh, UTl, n, true);
+    split_tf32(c, D, n, n, n, Xi, scratch, n);            // Uq hi, lo
+    split_tf32(c, D, n, n, n, UTl, Fs, n, true);          // Uq^T hi, lo
     launch_invert_perm(c, perm, n);
   }
   for (int l = 0; l < count; ++l) {
-    // QEP applied in processing order: W'P = WP + 2 alpha ((G P) U^T) U
+    // QEP applied in processing order: W'P = WP + 2 alpha ((G P) Uq^T) Uq.
+    // QEP makes no dead-column fix: a dead column's correction is zero (its
+    // column of d is), so W' keeps W there; GPTQ zeroes it below.
+    PhaseScope ps(c, kPhQepApply);
+    launch_permute_w(c, Gl(l), m[l], n, perm, nullptr, Wp);          // G P
+    split_tf32(c, Wp, m[l], n, n, Ph, Pl, n);
+    gemm_tf32x3(c, m[l], n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, Gl(l), n, kBLower);  // T = (G P) Uq^T
+    split_tf32(c, Gl(l), m[l], n, n, Ph, Pl, n);
+    launch_permute_w(c, W[l], m[l], n, perm, nullptr, Wp);           // W P
+    gemm_tf32x3(c, m[l], n, n, 2.f * alpha, Ph, Pl, n, UTl, Fs, n, true, Wp, n, kBUpper);
+    launch_permute_w(c, Wp, m[l], n, perm + n, nullptr, W_out[l]);   // back to original order
+  }
+  {
+    // GPTQ with its own factor U (in UTh): U^T split for the trailing updates
+    PhaseScope ps(c, kPhGptqPrep);
+    split_tf32(c, UTh, n, n, n, Xi, scratch, n, true);
+  }
+  for (int l = 0; l < count; ++l) {
     {
-      PhaseScope ps(c, kPhQepApply);
-      launch_permute_w(c, Gl(l), m[l], n, perm, dead, Wp);             // G P
-      split_tf32(c, Wp, m[l], n, n, Ph, Pl, n);
-      gemm_tf32x3(c, m[l], n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, Gl(l), n, kBLower);  // T = (G P) U^T
-      split_tf32(c, Gl(l), m[l], n, n, Ph, Pl, n);
-      launch_permute_w(c, W[l], m[l], n, perm, dead, Wp);              // W P
-      gemm_tf32x3(c, m[l], n, n, 2.f * alpha, Ph, Pl, n, UTh, UTl, n, true, Wp, n, kBUpper);
-      launch_permute_w(c, Wp, m[l], n, perm + n, dead, W_out[l]);      // back to original order
+      // GPTQ's working copy: W' in processing order, dead columns zeroed
+      PhaseScope ps(c, kPhGptqPrep);
+      launch_permute_w(c, W_out[l], m[l], n, perm, dead, Wp);
     }
     if (act_order) {
       PhaseScope ps(c, kPhGptqPrep);
       launch_static_grid(c, W_out[l], m[l], n, static_cast<int>(G), wbits, dead, scales[l], zeros[l]);
     }
-    gptq_sweep_and_pack(c, Wp, m[l], n, D, UTh, UTl, static_cast<int>(G), wbits, act_order != 0, perm, scales[l],
-                        zeros[l], codes8, Errh, Errl, codes[l], l == 0 ? perm_out : nullptr);
+    gptq_sweep_and_pack(c, Wp, m[l], n, UTh, Xi, scratch, static_cast<int>(G), wbits, act_order != 0, perm,
+                        scales[l], zeros[l], codes8, Errh, Errl, codes[l], l == 0 ? perm_out : nullptr);
   }
   return finish(c);
 }
@@ -579,6 +566,7 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
     sizing.take<float>(nn + 4096);                // recursion scratch of the side-stream factorisation
     sizing.take<float>(factor_split_floats(n));   // split copies inside the factorisation
     sizing.take<DiagStats>(1);
+    sizing.take<int>(1);                          // W's tf32 lo-half flag
     const size_t cross_bytes = cross_scratch_bytes(n_tok, n);
     sizing.take<unsigned char>(cross_bytes);      // the cross product's operands
     Carve cv{workspace(c, sizing.off + 256)};
@@ -594,6 +582,7 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
     float* Fs = cv.take<float>(nn + 4096);
     float* fsplit = cv.take<float>(factor_split_floats(n));
     DiagStats* stats = cv.take<DiagStats>(1);
+    int* lo_flag = cv.take<int>(1);
     unsigned char* cross_scratch = cv.take<unsigned char>(cross_bytes);
 
     const float* Hp = H_opt;
@@ -631,8 +620,8 @@ int oc_qep_correct(const float* W, int64_t m, int64_t n, const void* X, const vo
       // G = W d on the tensor cores (3xTF32 from split operands)
       PhaseScope ps(c, kPhQepWDelta);
       split_tf32(c, D, n, n, n, Xi, scratch, n, true);  // d^T: B operands are stored [N x K]
-      split_tf32(c, W, m, n, n, Ph, Pl, n);
-      gemm_tf32x3(c, m, n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, G, n, kANone);
+      split_tf32(c, W, m, n, n, Ph, Pl, n, false, lo_flag);
+      gemm_tf32x3(c, m, n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, G, n, kANone, lo_flag);
     }
     check_cuda(cudaStreamWaitEvent(c.stream, ss.join, 0), "cudaStreamWaitEvent(join)");
     {
@@ -672,8 +661,8 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
     sizing.take<float>(nn + 4096);     // recursion scratch -> U_lo
     sizing.take<float>(mn);            // Wp
     sizing.take<unsigned char>(mn);    // codes8
-    sizing.take<float>(static_cast<size_t>(m) * 128);  // Err_hi
-    sizing.take<float>(static_cast<size_t>(m) * 128);  // Err_lo
+    sizing.take<float>(static_cast<size_t>(m) * kSuperBlock);  // superblock errors, hi
+    sizing.take<float>(static_cast<size_t>(m) * kSuperBlock);  // and lo
     sizing.take<int32_t>(2 * static_cast<size_t>(n));  // perm | inverse
     sizing.take<unsigned char>(n);     // dead
     sizing.take<float>(factor_split_floats(n));  // split copies inside the factorisation
@@ -684,8 +673,8 @@ int oc_gptq_quantize(const float* W, int64_t m, int64_t n, const float* H, int w
     float* scratch = cv.take<float>(nn + 4096);
     float* Wp = cv.take<float>(mn);
     unsigned char* codes8 = cv.take<unsigned char>(mn);
-    float* Errh = cv.take<float>(static_cast<size_t>(m) * 128);
-    float* Errl = cv.take<float>(static_cast<size_t>(m) * 128);
+    float* Errh = cv.take<float>(static_cast<size_t>(m) * kSuperBlock);
+    float* Errl = cv.take<float>(static_cast<size_t>(m) * kSuperBlock);
     int32_t* perm = cv.take<int32_t>(2 * static_cast<size_t>(n));
     unsigned char* dead = cv.take<unsigned char>(n);
     float* fsplit = cv.take<float>(factor_split_floats(n));

@@ -157,16 +157,21 @@ void gemm_f32(const Ctx& c, bool tA, bool tB, int64_t M, int64_t N, int64_t K, f
 // x_hi = tf32(x), x_lo = tf32(x - x_hi) of a rows x cols block of src
 // (leading dimension lds); written untransposed (ldd) or, with transpose,
 // as the cols x rows transpose (ldd = leading dimension of the transpose).
+// lo_nz (untransposed, 16-byte aligned rows only): a device flag set to 1 if
+// any lo is non-zero, else 0 (x exact in tf32).
 void split_tf32(const Ctx& c, const float* src, int64_t rows, int64_t cols, int64_t lds, float* hi,
-                float* lo, int64_t ldd, bool transpose = false);
+                float* lo, int64_t ldd, bool transpose = false, int* lo_nz = nullptr);
 
 // fp32-accurate tensor-core GEMM from split operands: C (+)= alpha A B^T with
 // A [M x K] (lda) and B [N x K] (ldb) row-major; accumulate selects C += over
 // C =.  Flags describe the triangles of A and of op(B) = B^T.  Pointers and
 // leading dimensions must allow 16-byte aligned TMA rows.
+// a_lo_nz, b_lo_nz: optional device flags from split_tf32; when one reads 0
+// that operand's lo half is all zero and its correction product is skipped.
 void gemm_tf32x3(const Ctx& c, int64_t M, int64_t N, int64_t K, float alpha, const float* A_hi,
                  const float* A_lo, int64_t lda, const float* B_hi, const float* B_lo, int64_t ldb,
-                 bool accumulate, float* C, int64_t ldc, unsigned flags);
+                 bool accumulate, float* C, int64_t ldc, unsigned flags, const int* a_lo_nz = nullptr,
+                 const int* b_lo_nz = nullptr);
 
 // U = upper Cholesky factor of (H_prepared)^-1, where H_prepared is formed by
 // `launch_build_reversed` into M (consumed).  Scratch must hold n*n/2 + 4096
@@ -195,15 +200,28 @@ void launch_identity_perm(const Ctx& c, int64_t n, int32_t* perm);
 void launch_build_reversed(const Ctx& c, const float* H, int64_t n, const int32_t* perm,
                            const DiagStats* stats, float hscale, bool fix_dead, float* M);
 
+// QEP's inverse factor in GPTQ's processing order, decided on the device:
+// when GPTQ's preparation (stats_g) found dead columns, QEP's own matrix
+// H + lam I (lam = stats_q->lam, no dead-column fix) permuted by perm is
+// factored into Uq (X, scratch, split: the factorisation's scratch);
+// otherwise the two dampened matrices are the same and Uq = Ug.  Recorded
+// once per (n, buffers) as a graph with a conditional node; no host read.
+void qep_factor_select(const Ctx& c, const float* H, int64_t n, const int32_t* perm, const DiagStats* stats_g,
+                       const DiagStats* stats_q, const float* Ug, float* Uq, float* X, float* scratch, float* split);
+
 // GPTQ pieces.
 void launch_permute_w(const Ctx& c, const float* W, int64_t m, int64_t n, const int32_t* perm,
                       const unsigned char* dead, float* Wp);
 void launch_static_grid(const Ctx& c, const float* W, int64_t m, int64_t n, int G, int wbits,
                         const unsigned char* dead, float* scales, float* zeros);
+// Err (and Err_lo) rows have err_ld floats (>= 128); the block's errors go to
+// their first 128 columns.
 void launch_sweep_block(const Ctx& c, float* Wp, int64_t m, int64_t n, const float* U,
                         int64_t j1, int G, int wbits, bool static_groups, const int32_t* perm,
                         float* scales, float* zeros, unsigned char* codes8, float* Err,
-                        float* Err_lo = nullptr);
+                        float* Err_lo = nullptr, int64_t err_ld = 128);
+// GPTQ's lazy updates: superblocks of this many columns (four sweep blocks).
+constexpr int64_t kSuperBlock = 512;
 // Packs codes8 (processing order) into the original-order bitstream; perm2
 // holds the processing order in its first n entries and receives the inverse
 // permutation in the next n.

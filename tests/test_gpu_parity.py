@@ -380,6 +380,36 @@ def test_fused_layer_matches_oracle(m, n, n_tok, wbits, G, act, dead, big):
     assert ident >= code_frac_for(cg.size), (ident, st)
 
 
+def test_fused_layer_async_returns_before_its_stream_finishes():
+    # In asynchronous mode the fused call only enqueues work: no step of it
+    # (not the dead-column decision either) waits for the device.  A spinning
+    # kernel ahead of it keeps the stream busy for about a second; the call
+    # must return while the stream still runs, and its results must equal a
+    # synchronous call's.
+    m, n, G = 256, 512, 128
+    L = random_layer_host(m, n, 2048, seed=3500)
+    W, X, Xh = dev(L["W"]), bf16_dev(L["X"]), bf16_dev(L["Xhat"])
+    ref = oc.oc_quantize_layer(W, X, Xh, 0.5, 0.01, 4, G, True)   # synchronous; sets up workspace and graphs
+    torch.cuda.synchronize()
+    out = dict(H=torch.empty(n, n, device="cuda"), W_out=torch.empty_like(W),
+               codes=torch.empty(m, n * 4 // 32, dtype=torch.int32, device="cuda"),
+               scales=torch.empty(m, n // G, device="cuda"), zeros=torch.empty(m, n // G, device="cuda"))
+    stream = torch.cuda.current_stream()
+    oc.oc_set_sync(False)
+    try:
+        torch.cuda._sleep(int(2e9))
+        oc.oc_quantize_layer(W, X, Xh, 0.5, 0.01, 4, G, True, **out)
+        busy = not stream.query()
+        status = oc.oc_stream_status(stream)
+    finally:
+        oc.oc_set_sync(True)
+    assert busy, "the call waited for its stream"
+    assert status == oc.OC_OK
+    assert torch.allclose(out["W_out"], ref[1], rtol=0, atol=1e-6 * float(ref[1].abs().max()))
+    assert float((out["codes"] == ref[2]).float().mean()) >= 0.99
+    assert torch.allclose(out["scales"], ref[3], rtol=1e-5, atol=0)
+
+
 # ----------------------------------------------------------------------------- layer groups
 
 @pytest.mark.parametrize("ms,n,n_tok,wbits,G,act,dead", [
