@@ -95,6 +95,16 @@ const char* oc_profile_phase_name(int phase);
 /* Kernel launches made by this library since it was loaded. */
 int64_t oc_launch_count(void);
 
+/* Test of the failure path (no counterpart in the method).  The next launch of
+ * the tensor-core product behind oc_hessian_accumulate, oc_qep_correct,
+ * oc_qep_terms and the fused calls has one thread per CTA wait on an
+ * on-device barrier that nothing releases.  That bounded wait gives up after
+ * its limit (2 s), records OC_ERR_TIMEOUT in the status word and stops the
+ * kernel before it issues any copy or MMA, so the call returns
+ * OC_ERR_TIMEOUT (synchronous mode) with its outputs not computed, and the
+ * device stays usable for the next call.  One-shot. */
+int oc_test_inject_stall(void);
+
 /*
  * Hessian accumulation:  H += 2 * X^T X   (n x n, fp32)
  *

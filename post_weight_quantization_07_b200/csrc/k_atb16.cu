@@ -102,6 +102,7 @@ struct Params {
   int* status;
   int mode;
   const int* flag;       // kBf16IfFlag
+  int stall;             // test of the failure path: stall on a barrier nothing releases
   const float* isc;      // kScaledF16: 1 / s_j, isc_n entries
   int64_t isc_n;
   // operand pass of the next token slice (xcount = 0: none): xcount 16-byte
@@ -221,7 +222,8 @@ atb16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ C
   uint64_t* tfull = bars + 2 * STAGES;   // [2], accumulator ready (this CTA's TMEM half)
   uint64_t* tempty = tfull + 2;          // [2], used in the leader: both epilogues done
   uint64_t* drain = tempty + 2;          // [1], all MMAs finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* stall_bar = drain + 1;       // [1], never arrived on (the test stall)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stall_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   // the same decision in every thread of every CTA, before any barrier
@@ -243,6 +245,7 @@ atb16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ C
       mbar_init(&tempty[a], 2 * EPI_WARPS);
     }
     mbar_init(drain, 1);
+    mbar_init(stall_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&mapA);
@@ -260,6 +263,18 @@ atb16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  if (p.stall) {
+    // Test of the failure path: one thread waits on a barrier that nothing
+    // arrives on.  The bounded wait gives up, records OC_ERR_TIMEOUT and
+    // raises the abort flag before any copy or MMA is issued, so every role
+    // below stops at its first wait and the kernel winds down normally.
+    if (threadIdx.x == 0 && !mbar_wait(stall_bar, 0)) {
+      record_error(p.status, kDevTimeout);
+      *abort_flag = 1;
+    }
+    __syncthreads();
+  }
+
   const int64_t stages_total = (p.n_tok + BK - 1) / BK;
 
   if (warp == 0) {
@@ -276,7 +291,7 @@ atb16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ C
         const int s = static_cast<int>(issued % STAGES);
         const uint32_t ph = static_cast<uint32_t>((issued / STAGES) & 1);
         int w = 1;
-        if (lane == 0) w = mbar_wait(&empty[s], ph ^ 1) && !*abort_flag;
+        if (lane == 0) w = mbar_wait_or_abort(&empty[s], ph ^ 1, abort_flag) && !*abort_flag;
         w = __shfl_sync(0xffffffffu, w, 0);
         if (!w) { ok = false; break; }
         if (lane == 0) {
@@ -328,7 +343,7 @@ atb16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ C
         const int64_t ks1 = ::min((int64_t)stages_total, ks0 + p.kc_stages);
         const int acc = it & 1;
         int w = 1;
-        if (lane == 0) w = mbar_wait(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1));
+        if (lane == 0) w = mbar_wait_or_abort(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1), abort_flag);
         w = __shfl_sync(0xffffffffu, w, 0);
         if (!w) { ok = false; break; }
         tc_fence_after();
@@ -337,7 +352,7 @@ atb16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ C
           const int s = static_cast<int>(consumed % STAGES);
           const uint32_t ph = static_cast<uint32_t>((consumed / STAGES) & 1);
           w = 1;
-          if (lane == 0) w = mbar_wait(&full[s], ph) && !*abort_flag;
+          if (lane == 0) w = mbar_wait_or_abort(&full[s], ph, abort_flag) && !*abort_flag;
           w = __shfl_sync(0xffffffffu, w, 0);
           if (!w) { ok = false; break; }
           tc_fence_after();
@@ -388,7 +403,7 @@ atb16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ C
       decode_tile(p, static_cast<int>(u % p.n_tiles), ti, tj);
       const int acc = it & 1;
       int w = 1;
-      if (lane == 0) w = mbar_wait(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1)) && !*abort_flag;
+      if (lane == 0) w = mbar_wait_or_abort(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1), abort_flag) && !*abort_flag;
       w = __shfl_sync(0xffffffffu, w, 0);
       if (!w) { ok = false; break; }
       tc_fence_after();
@@ -526,6 +541,14 @@ __global__ void column_scales_kernel(const float* __restrict__ H, int64_t n, flo
 
 namespace {
 
+bool g_stall_request = false;  // guarded by the library lock, like every launch
+
+bool take_stall_request() {
+  const bool r = g_stall_request;
+  g_stall_request = false;
+  return r;
+}
+
 // One token slice's operand pass for the fused launch (or a standalone one).
 struct SlicePass {
   const void* X;
@@ -615,6 +638,7 @@ void launch_atb16_ex(const Ctx& c, const void* A, const void* B, int64_t n_tok, 
   p.status = c.status;
   p.mode = mode;
   p.flag = flag;
+  p.stall = take_stall_request() ? 1 : 0;
   p.isc = isc;
   p.isc_n = std::max(M, N);
   const int64_t clusters = std::min<int64_t>(p.units, clusters_avail);
@@ -640,6 +664,8 @@ void launch_atb16_ex(const Ctx& c, const void* A, const void* B, int64_t n_tok, 
 }
 
 }  // namespace
+
+void request_test_stall() { g_stall_request = true; }
 
 void launch_atb16(const Ctx& c, const void* A, const void* B, int64_t n_tok, int64_t M, int64_t N, float alpha,
                   float* C, int64_t ldc, bool upper_only, int max_ctas) {

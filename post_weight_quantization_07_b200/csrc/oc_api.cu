@@ -499,6 +499,13 @@ const char* oc_profile_phase_name(int phase) { return phase_name(phase); }
 
 int64_t oc_launch_count(void) { return launch_count(); }
 
+int oc_test_inject_stall(void) {
+  return guarded([&]() -> int {
+    request_test_stall();
+    return OC_OK;
+  });
+}
+
 int oc_workspace_release(void) {
   return guarded([&]() -> int {
     int dev = 0;

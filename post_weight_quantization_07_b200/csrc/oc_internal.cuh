@@ -109,6 +109,10 @@ CUtensorMap make_tmap_2d(const void* base, CUtensorMapDataType dt, int elem_byte
 void launch_atb16(const Ctx& c, const void* A, const void* B, int64_t n_tok, int64_t M, int64_t N, float alpha,
                   float* C, int64_t ldc, bool upper_only, int max_ctas = 0);
 
+// The next launch_atb16 / launch_cross_product launch of the tensor-core
+// product stalls on a barrier nothing releases (test of the failure path).
+void request_test_stall();
+
 // QEP's cross term d = (X - Xhat)^T Xhat (n x n, fp32, overwritten) from the
 // bf16 token-major pair X, Xhat [n_tok x n] and H = 2 Xhat^T Xhat of the same
 // tokens (its diagonal sets per-feature fp16 scales).  Runs as `parts` token

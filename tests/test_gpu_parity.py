@@ -68,6 +68,21 @@ def test_hessian_matches_oracle(n, n_tok):
     assert np.array_equal(Hg, Hg.T)
 
 
+def test_bounded_wait_runs_out_and_the_library_recovers():
+    # A barrier nothing releases (oc_test_inject_stall): the kernel's bounded
+    # wait gives up, the call reports OC_ERR_TIMEOUT, and the next call runs
+    # normally on the same device.
+    L = random_layer_host(8, 256, 1000, seed=104)
+    H = dev(np.zeros((256, 256)))
+    oc.oc_test_inject_stall()
+    with pytest.raises(oc.OcError) as e:
+        oc.oc_hessian_accumulate(bf16_dev(L["Xhat"]), H)
+    assert e.value.status == oc.OC_ERR_TIMEOUT
+    assert oc.oc_stream_status(None) == oc.OC_OK   # the error was collected once
+    Hg = gpu_hessian(L["Xhat"])
+    assert rel_fro(Hg, oracle.hessian(L["Xhat"])) <= H_TOL
+
+
 def test_hessian_accumulates_and_ignores_empty():
     L = random_layer_host(8, 256, 1500, seed=7)
     H1 = gpu_hessian(L["Xhat"][:700])
