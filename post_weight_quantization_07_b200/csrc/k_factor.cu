@@ -14,7 +14,7 @@
 //                Y = L21 X11                               (GEMM, before the next recursion)
 //                L22 = chol(A22'), X22 = L22^-1            (recurse)
 //                X21 = -X22 Y                              (GEMM)
-// with 128x128 leaves factored and inverted inside one CTA.
+// with 128x128 leaves that go straight to X = L^-1 inside one CTA.
 #include <algorithm>
 #include <cmath>
 #include <vector>
@@ -138,262 +138,144 @@ __global__ void build_reversed_kernel(const float* __restrict__ H, int64_t n,
 // ---------------------------------------------------------------- leaf
 // Cholesky of an s x s (s <= 128) diagonal block at M (lower part read) and
 // the inverse of its factor, written to X (lower, explicit zeros above), in
-// one CTA with the whole block in shared memory.  The block is split
-// recursively, 128 -> 64 -> 32, with the same four products as the outer
-// recursion:
-//   X11 = L11^-1 (recurse);  T = A21 X11^T (= L21);  A22 -= T T^T;
-//   Y = T X11;  X22 = L22^-1 (recurse);  X21 = -X22 Y.
-// A 32x32 block is factored and inverted by one warp: lane i holds row i in
-// registers; column k of L reaches the other lanes by shuffles; the inverse is
-// forward substitution per column (lane j owns column j of X) reading L from
-// shared memory.  Rows and columns beyond s are padded with the identity.
-constexpr int LDA = LEAF + 1;      // padded leading dimensions (bank spread)
-constexpr int LDT = LEAF / 2 + 1;
+// one CTA with the block in shared memory.  Rows and columns beyond s are
+// padded with the identity.
+//
+// One array S holds both: before step K its columns < K hold rows of
+// X = L^-1 and its columns >= K the Cholesky trailing matrix.  Step K takes
+// the 4 x 4 pivot block P = S[K:K+4, K:K+4], factors it, P = L_p L_p^T, and
+// inverts the factor, Z = L_p^-1 (every thread, in registers), then forms one
+// 4-vector per index j:
+//   v_j = Z S[K:K+4, j]   (j < K: the final rows K..K+3 of X at column j),
+//   v_j = Z[:, j - K]     (K <= j < K+4: the pivot block of X),
+//   v_j = Z S[j, K:K+4]   (j >= K+4: row j of L's column block),
+// stores the first two kinds as rows K..K+3 of X (final from here on), clears
+// the column block below the pivot, and applies
+//   S_ij -= v_i . v_j   for every i >= K+4 and j <= i,
+// which is at once the trailing update A_ij -= L_i,K:K+4 L_j,K:K+4 (j >= K+4),
+// the new columns X_i,K:K+4 = -L_i,K:K+4 Z (K <= j < K+4) and the row
+// operation that applies the inverse of step K's elementary factor to the
+// rows of X (j < K).  So the leaf is 32 rank-4 steps, each two barriers apart,
+// with all threads sharing the update of the rows below the pivot: a warp per
+// row, and each lane keeps the same four columns (and their 4-vectors, loaded
+// once per step) for every row, so a row costs one broadcast load and one
+// load and store per 32 columns of shared memory.
+constexpr int LDS = LEAF + 1;      // padded row (bank spread for the column reads)
+constexpr int LEAF_THREADS = 512;
+constexpr int PB = 4;              // pivot block
+constexpr size_t LEAF_SMEM = static_cast<size_t>(LEAF) * LDS * sizeof(float) + LEAF * sizeof(float4);
 
-struct LeafSmem {
-  float4 col4[32];                 // 4 columns of the current 32 block, one row per lane
-  float4 blk[4];                   // the current 4x4 pivot block
-  float A[LEAF * LDA];
-  float X[LEAF * LDA];
-  float T[(LEAF / 2) * LDT];       // L21 of the 128 level; temporaries of the 64 level
-  float Y[(LEAF / 2) * LDT];       // Y of the 128 level (lives across the right half)
-  float L32[32 * 33];              // factor of the current 32 block
-  float R32[32];                   // reciprocals of its diagonal
-};
-
-// One step of the 32x32 factor: columns K..K+3.  The 4x4 pivot block is
-// factored redundantly by every lane in registers; each lane then finishes its
-// own row's four entries, and the four columns reach the other lanes as one
-// float4 per row through shared memory.
-template <int K>
-__device__ __forceinline__ void chol32_step(LeafSmem& sm, float (&a)[32], int lane, bool& bad) {
-  if (lane >= K && lane < K + 4) sm.blk[lane - K] = make_float4(a[K], a[K + 1], a[K + 2], a[K + 3]);
-  __syncwarp();
-  const float4 q0 = sm.blk[0], q1 = sm.blk[1], q2 = sm.blk[2], q3 = sm.blk[3];
-  const float r0 = rsqrtf(q0.x);
-  const float l10 = q1.x * r0, l20 = q2.x * r0, l30 = q3.x * r0;
-  const float d1 = fmaf(-l10, l10, q1.y);
-  const float r1 = rsqrtf(d1);
-  const float l21 = fmaf(-l20, l10, q2.y) * r1, l31 = fmaf(-l30, l10, q3.y) * r1;
-  const float d2 = fmaf(-l21, l21, fmaf(-l20, l20, q2.z));
-  const float r2 = rsqrtf(d2);
-  const float l32 = fmaf(-l31, l21, fmaf(-l30, l20, q3.z)) * r2;
-  const float d3 = fmaf(-l32, l32, fmaf(-l31, l31, fmaf(-l30, l30, q3.w)));
-  const float r3 = rsqrtf(d3);
-  if (!(q0.x > 0.f) || !(d1 > 0.f) || !(d2 > 0.f) || !(d3 > 0.f) || !isfinite(q0.x + d1 + d2 + d3)) bad = true;
-  const float x0 = a[K] * r0;
-  const float x1 = fmaf(-x0, l10, a[K + 1]) * r1;
-  const float x2 = fmaf(-x1, l21, fmaf(-x0, l20, a[K + 2])) * r2;
-  const float x3 = fmaf(-x2, l32, fmaf(-x1, l31, fmaf(-x0, l30, a[K + 3]))) * r3;
-  const int rr = lane - K;  // rows of the pivot block keep zeros above the diagonal
-  a[K] = x0;
-  a[K + 1] = (rr >= 0 && rr < 1) ? 0.f : x1;
-  a[K + 2] = (rr >= 0 && rr < 2) ? 0.f : x2;
-  a[K + 3] = (rr >= 0 && rr < 3) ? 0.f : x3;
-  if constexpr (K + 4 < 32) {
-    sm.col4[lane] = make_float4(a[K], a[K + 1], a[K + 2], a[K + 3]);
-    __syncwarp();
-#pragma unroll
-    for (int j = K + 4; j < 32; ++j) {
-      const float4 v = sm.col4[j];
-      if (lane >= j)
-        a[j] = fmaf(-a[K + 3], v.w, fmaf(-a[K + 2], v.z, fmaf(-a[K + 1], v.y, fmaf(-a[K], v.x, a[j]))));
-    }
-    chol32_step<K + 4>(sm, a, lane, bad);
-  }
-}
-
-__device__ __noinline__ void warp_chol_inv32(LeafSmem& sm, int off, int* status) {
-  const int lane = threadIdx.x & 31;
-  float a[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) a[j] = (j <= lane) ? sm.A[(off + lane) * LDA + off + j] : 0.f;
-  bool bad = false;
-  chol32_step<0>(sm, a, lane, bad);
-  if (bad && lane == 0) record_error(status, kDevNotSpd);
-  float dl = 1.f;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    sm.L32[lane * 33 + j] = a[j];
-    if (j == lane) dl = a[j];
-  }
-  sm.R32[lane] = 1.f / dl;
-  __syncwarp();
-  // Column `lane` of X = L^-1 by right-looking forward substitution: at step k
-  // x_k = b_k / L_kk, then every later row takes b_i -= L_ik x_k (independent
-  // updates: the dependent chain is one multiply and one FMA per step).
-  float b[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) b[i] = (i == lane) ? 1.f : 0.f;
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    const float xk = b[k] * sm.R32[k];
-    b[k] = xk;
-#pragma unroll
-    for (int i = k + 1; i < 32; ++i) b[i] = fmaf(-sm.L32[i * 33 + k], xk, b[i]);
-  }
-#pragma unroll
-  for (int i = 0; i < 32; ++i) sm.X[(off + i) * LDA + off + lane] = b[i];
-}
-
-// The four products of one recursion node of half width H inside the CTA
-// (256 threads, each a TR x TC register tile of the H x H outputs).
-template <int H>
-__device__ __forceinline__ void node_pre(LeafSmem& sm, int off, float* T, int ldt, float* Y, int ldy) {
-  constexpr int TR = (H == 64) ? 4 : 2, TC = TR;
-  constexpr int NTC = H / TC;
-  const int t = threadIdx.x;
-  const int i0 = (t / NTC) * TR, j0 = (t % NTC) * TC;
-  const float* A21 = &sm.A[(off + H) * LDA + off];
-  float* A22 = &sm.A[(off + H) * LDA + off + H];
-  const float* X11 = &sm.X[off * LDA + off];
-  // T = A21 X11^T: T[i][j] = sum_{k <= j} A21[i][k] X11[j][k]
-  {
-    float acc[TR][TC] = {};
-    for (int k = 0; k < j0 + TC; ++k) {
-      float av[TR], bv[TC];
-#pragma unroll
-      for (int r = 0; r < TR; ++r) av[r] = A21[(i0 + r) * LDA + k];
-#pragma unroll
-      for (int c = 0; c < TC; ++c) bv[c] = X11[(j0 + c) * LDA + k];
-#pragma unroll
-      for (int r = 0; r < TR; ++r)
-#pragma unroll
-        for (int c = 0; c < TC; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
-    }
-#pragma unroll
-    for (int r = 0; r < TR; ++r)
-#pragma unroll
-      for (int c = 0; c < TC; ++c) T[(i0 + r) * ldt + j0 + c] = acc[r][c];
-  }
-  __syncthreads();
-  // A22 -= T T^T (tiles touching the lower triangle)
-  if (j0 <= i0 + TR - 1) {
-    float acc[TR][TC] = {};
-    for (int k = 0; k < H; ++k) {
-      float av[TR], bv[TC];
-#pragma unroll
-      for (int r = 0; r < TR; ++r) av[r] = T[(i0 + r) * ldt + k];
-#pragma unroll
-      for (int c = 0; c < TC; ++c) bv[c] = T[(j0 + c) * ldt + k];
-#pragma unroll
-      for (int r = 0; r < TR; ++r)
-#pragma unroll
-        for (int c = 0; c < TC; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
-    }
-#pragma unroll
-    for (int r = 0; r < TR; ++r)
-#pragma unroll
-      for (int c = 0; c < TC; ++c) A22[(i0 + r) * LDA + j0 + c] -= acc[r][c];
-  }
-  // Y = T X11: Y[i][j] = sum_{k >= j} T[i][k] X11[k][j]
-  {
-    float acc[TR][TC] = {};
-    for (int k = j0; k < H; ++k) {
-      float av[TR], bv[TC];
-#pragma unroll
-      for (int r = 0; r < TR; ++r) av[r] = T[(i0 + r) * ldt + k];
-#pragma unroll
-      for (int c = 0; c < TC; ++c) bv[c] = X11[k * LDA + j0 + c];
-#pragma unroll
-      for (int r = 0; r < TR; ++r)
-#pragma unroll
-        for (int c = 0; c < TC; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
-    }
-#pragma unroll
-    for (int r = 0; r < TR; ++r)
-#pragma unroll
-      for (int c = 0; c < TC; ++c) Y[(i0 + r) * ldy + j0 + c] = acc[r][c];
-  }
-  __syncthreads();
-}
-
-template <int H>
-__device__ __forceinline__ void node_post(LeafSmem& sm, int off, const float* Y, int ldy) {
-  constexpr int TR = (H == 64) ? 4 : 2, TC = TR;
-  constexpr int NTC = H / TC;
-  const int t = threadIdx.x;
-  const int i0 = (t / NTC) * TR, j0 = (t % NTC) * TC;
-  const float* X22 = &sm.X[(off + H) * LDA + off + H];
-  float* X21 = &sm.X[(off + H) * LDA + off];
-  // X21 = -X22 Y: X21[i][j] = -sum_{k <= i} X22[i][k] Y[k][j]
-  float acc[TR][TC] = {};
-  for (int k = 0; k < i0 + TR; ++k) {
-    float av[TR], bv[TC];
-#pragma unroll
-    for (int r = 0; r < TR; ++r) av[r] = X22[(i0 + r) * LDA + k];
-#pragma unroll
-    for (int c = 0; c < TC; ++c) bv[c] = Y[k * ldy + j0 + c];
-#pragma unroll
-    for (int r = 0; r < TR; ++r)
-#pragma unroll
-      for (int c = 0; c < TC; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
-  }
-#pragma unroll
-  for (int r = 0; r < TR; ++r)
-#pragma unroll
-    for (int c = 0; c < TC; ++c) X21[(i0 + r) * LDA + j0 + c] = -acc[r][c];
-  __syncthreads();
-}
-
-__device__ __forceinline__ void leaf32(LeafSmem& sm, int off, int* status) {
-  if ((threadIdx.x >> 5) == 0) warp_chol_inv32(sm, off, status);
-  __syncthreads();
-}
-
-// 64 block at `off`; its temporaries live in sm.T (T at 0, Y at 32 rows on).
-__device__ __forceinline__ void leaf64(LeafSmem& sm, int off, int* status) {
-  float* T = sm.T;
-  float* Y = sm.T + 32 * 33;
-  leaf32(sm, off, status);
-  node_pre<32>(sm, off, T, 33, Y, 33);
-  leaf32(sm, off + 32, status);
-  node_post<32>(sm, off, Y, 33);
-}
-
-__global__ void __launch_bounds__(256) leaf_chol_inv_kernel(const float* __restrict__ M, float* __restrict__ X,
-                                                            int64_t ld, int s, int* status) {
+__global__ void __launch_bounds__(LEAF_THREADS) leaf_chol_inv_kernel(const float* __restrict__ M,
+                                                                     float* __restrict__ X, int64_t ld, int s,
+                                                                     int* status) {
   extern __shared__ __align__(16) float leaf_smem[];
-  LeafSmem& sm = *reinterpret_cast<LeafSmem*>(leaf_smem);
+  float4* V = reinterpret_cast<float4*>(leaf_smem);              // [LEAF]
+  float* S = leaf_smem + 4 * LEAF;                               // [LEAF][LDS]
   const int t = threadIdx.x;
-  // Load the block with 16 independent 16-byte loads per thread in flight
-  // (rows of M are 16-byte aligned: n is a multiple of 64).
-  float4 v[16];
-#pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const int e4 = t + 256 * q;          // float4 index in the 128 x 128 block
-    const int i = e4 >> 5, j = (e4 & 31) * 4;
-    v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < s && j <= i && j < s) v[q] = *reinterpret_cast<const float4*>(M + static_cast<int64_t>(i) * ld + j);
-  }
-#pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const int e4 = t + 256 * q;
-    const int i = e4 >> 5, j = (e4 & 31) * 4;
-    const float vv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+  const int warp = t >> 5, lane = t & 31;
+  // Load: 16-byte loads (rows of M are 16-byte aligned: ld is a multiple of
+  // 64 and the block starts at a multiple of 128), lower part only.
+  for (int e4 = t; e4 < LEAF * LEAF / 4; e4 += LEAF_THREADS) {
+    const int i = e4 / (LEAF / 4), j = (e4 % (LEAF / 4)) * 4;
+    float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < s && j <= i && j < s) q = *reinterpret_cast<const float4*>(M + static_cast<int64_t>(i) * ld + j);
+    const float qq[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      float x = (j + c <= i && j + c < s) ? vv[c] : 0.f;
+      float x = (j + c <= i && j + c < s) ? qq[c] : 0.f;
       if (i >= s && i == j + c) x = 1.f;  // identity padding beyond s
-      sm.A[i * LDA + j + c] = x;
-      sm.X[i * LDA + j + c] = 0.f;
+      S[i * LDS + j + c] = x;
     }
   }
   __syncthreads();
-  leaf64(sm, 0, status);
-  node_pre<64>(sm, 0, sm.T, LDT, sm.Y, LDT);
-  leaf64(sm, 64, status);
-  node_post<64>(sm, 0, sm.Y, LDT);
+  bool bad = false;
+  for (int K = 0; K < LEAF; K += PB) {
+    if (t < LEAF) {
+      // P = L_p L_p^T and Z = L_p^-1 (lower 4 x 4), redundantly per thread
+      const float* P = S + K * LDS + K;
+      const float p00 = P[0];
+      const float p10 = P[LDS], p11 = P[LDS + 1];
+      const float p20 = P[2 * LDS], p21 = P[2 * LDS + 1], p22 = P[2 * LDS + 2];
+      const float p30 = P[3 * LDS], p31 = P[3 * LDS + 1], p32 = P[3 * LDS + 2], p33 = P[3 * LDS + 3];
+      const float r0 = rsqrtf(p00);
+      const float l10 = p10 * r0, l20 = p20 * r0, l30 = p30 * r0;
+      const float d1 = fmaf(-l10, l10, p11);
+      const float r1 = rsqrtf(d1);
+      const float l21 = fmaf(-l20, l10, p21) * r1, l31 = fmaf(-l30, l10, p31) * r1;
+      const float d2 = fmaf(-l21, l21, fmaf(-l20, l20, p22));
+      const float r2 = rsqrtf(d2);
+      const float l32 = fmaf(-l31, l21, fmaf(-l30, l20, p32)) * r2;
+      const float d3 = fmaf(-l32, l32, fmaf(-l31, l31, fmaf(-l30, l30, p33)));
+      const float r3 = rsqrtf(d3);
+      if (!(p00 > 0.f) || !(d1 > 0.f) || !(d2 > 0.f) || !(d3 > 0.f) || !isfinite(p00 + d1 + d2 + d3)) bad = true;
+      // Z = L_p^-1 by forward substitution (z_ii = r_i)
+      const float z00 = r0;
+      const float z10 = -l10 * r0 * r1, z11 = r1;
+      const float z20 = -fmaf(l21, z10, l20 * z00) * r2, z21 = -l21 * z11 * r2, z22 = r2;
+      const float z30 = -fmaf(l32, z20, fmaf(l31, z10, l30 * z00)) * r3;
+      const float z31 = -fmaf(l32, z21, l31 * z11) * r3, z32 = -l32 * z22 * r3, z33 = r3;
+      const int j = t;
+      float4 w;
+      if (j < K || j >= K + PB) {
+        float a0, a1, a2, a3;
+        if (j < K) {
+          a0 = S[K * LDS + j]; a1 = S[(K + 1) * LDS + j]; a2 = S[(K + 2) * LDS + j]; a3 = S[(K + 3) * LDS + j];
+        } else {
+          a0 = S[j * LDS + K]; a1 = S[j * LDS + K + 1]; a2 = S[j * LDS + K + 2]; a3 = S[j * LDS + K + 3];
+        }
+        w.x = z00 * a0;
+        w.y = fmaf(z11, a1, z10 * a0);
+        w.z = fmaf(z22, a2, fmaf(z21, a1, z20 * a0));
+        w.w = fmaf(z33, a3, fmaf(z32, a2, fmaf(z31, a1, z30 * a0)));
+        if (j < K) {
+          S[K * LDS + j] = w.x; S[(K + 1) * LDS + j] = w.y; S[(K + 2) * LDS + j] = w.z; S[(K + 3) * LDS + j] = w.w;
+        } else {
+          S[j * LDS + K] = 0.f; S[j * LDS + K + 1] = 0.f; S[j * LDS + K + 2] = 0.f; S[j * LDS + K + 3] = 0.f;
+        }
+      } else {
+        // column c = j - K of Z; rows K + c .. K + 3 of S take its lower part
+        const int c = j - K;
+        w = (c == 0) ? make_float4(z00, z10, z20, z30)
+          : (c == 1) ? make_float4(0.f, z11, z21, z31)
+          : (c == 2) ? make_float4(0.f, 0.f, z22, z32) : make_float4(0.f, 0.f, 0.f, z33);
+        const float wc[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const int e4 = t + 256 * q;
-    const int i = e4 >> 5, j = (e4 & 31) * 4;
+        for (int r = 0; r < PB; ++r)
+          if (r >= c) S[(K + r) * LDS + j] = wc[r];
+      }
+      V[j] = w;
+    }
+    __syncthreads();
+    {
+      // lane keeps columns j = lane + 32 q and their 4-vectors for the step
+      float4 vj[LEAF / 32];
+#pragma unroll
+      for (int q = 0; q < LEAF / 32; ++q) vj[q] = V[lane + 32 * q];
+      for (int i = K + PB + warp; i < LEAF; i += LEAF_THREADS / 32) {
+        const float4 vi = V[i];
+        float* row = S + i * LDS;
+        float x[LEAF / 32];
+#pragma unroll
+        for (int q = 0; q < LEAF / 32; ++q)
+          if (lane + 32 * q <= i) x[q] = row[lane + 32 * q];
+#pragma unroll
+        for (int q = 0; q < LEAF / 32; ++q)
+          if (lane + 32 * q <= i)
+            row[lane + 32 * q] =
+                fmaf(-vi.w, vj[q].w, fmaf(-vi.z, vj[q].z, fmaf(-vi.y, vj[q].y, fmaf(-vi.x, vj[q].x, x[q]))));
+      }
+    }
+    __syncthreads();
+  }
+  if (t == 0 && bad) record_error(status, kDevNotSpd);
+  for (int e4 = t; e4 < LEAF * LEAF / 4; e4 += LEAF_THREADS) {
+    const int i = e4 / (LEAF / 4), j = (e4 % (LEAF / 4)) * 4;
     if (i < s && j < s) {
       float4 o;
-      o.x = (j + 0 <= i) ? sm.X[i * LDA + j + 0] : 0.f;
-      o.y = (j + 1 <= i) ? sm.X[i * LDA + j + 1] : 0.f;
-      o.z = (j + 2 <= i) ? sm.X[i * LDA + j + 2] : 0.f;
-      o.w = (j + 3 <= i) ? sm.X[i * LDA + j + 3] : 0.f;
+      o.x = (j + 0 <= i) ? S[i * LDS + j + 0] : 0.f;
+      o.y = (j + 1 <= i) ? S[i * LDS + j + 1] : 0.f;
+      o.z = (j + 2 <= i) ? S[i * LDS + j + 2] : 0.f;
+      o.w = (j + 3 <= i) ? S[i * LDS + j + 3] : 0.f;
       *reinterpret_cast<float4*>(X + static_cast<int64_t>(i) * ld + j) = o;
     }
   }
@@ -439,11 +321,11 @@ void chol_inv_rec(const Ctx& c, float* M, float* X, int64_t ld, int64_t off, int
     static bool attr_done[64] = {false};
     if (!attr_done[c.device & 63]) {
       check_cuda(cudaFuncSetAttribute(leaf_chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(sizeof(LeafSmem))),
+                                      static_cast<int>(LEAF_SMEM)),
                  "cudaFuncSetAttribute(leaf)");
       attr_done[c.device & 63] = true;
     }
-    leaf_chol_inv_kernel<<<1, 256, sizeof(LeafSmem), c.stream>>>(Md, Xd, ld, static_cast<int>(s), c.status);
+    leaf_chol_inv_kernel<<<1, LEAF_THREADS, LEAF_SMEM, c.stream>>>(Md, Xd, ld, static_cast<int>(s), c.status);
     check_launch("leaf_chol_inv_kernel");
     return;
   }

@@ -135,7 +135,8 @@ constexpr int kSideSMs = 8;
 // Most layers one oc_quantize_layer_group call takes.
 constexpr int kMaxGroup = 16;
 // The cross product beside it runs as up to kCrossParts launches over token
-// ranges of at least kCrossPartMinTokens tokens each.
+// ranges of at least kCrossPartMinTokens tokens each: each boundary lets the
+// factorisation's pending products take the whole GPU.
 constexpr int64_t kCrossParts = 32;
 constexpr int64_t kCrossPartMinTokens = 8192;
 
