@@ -438,6 +438,10 @@ def teacher_forced_check(W, H, wbits: int, groupsize: int, damp: float, act_orde
     m, n = W.shape
     maxq = (1 << wbits) - 1
     G = _group_size(groupsize, n)
+    if not act_order and not (block % G == 0 or G % block == 0 or G == n):
+        # the same constraint as gptq_sweep: a dynamic group's values are read
+        # at its first column, so it must not start inside a block and run past it
+        raise ValueError("groupsize must divide the block or be a multiple of it")
     prep = gptq_prepare(W, H, damp, act_order, perm=perm)
     perm = prep["perm"]
     U = inv_chol_upper(prep["Hd"]) if U is None else _f64(U)

@@ -97,6 +97,8 @@ struct Params {
   int tiles_i, tiles_j, n_tiles;
   int kc_stages, n_kc;
   int64_t units;
+  int64_t full_units;    // units [0, full_units) are whole chunks
+  int split_k;           // each later unit is one of split_k parts of a chunk
   int upper_only;
   float alpha;
   int* status;
@@ -208,6 +210,25 @@ __device__ __forceinline__ void decode_tile(const Params& p, int tile, int& ti, 
   ti = t;
 }
 
+// Unit u -> output tile and token stages [ks0, ks1).  Units are chunk-major
+// (the clusters of one round stream the same token window through L2).  The
+// chunks that would form a last, partly filled round are cut into split_k
+// parts, so that the last round spreads over every cluster.
+__device__ __forceinline__ void decode_unit(const Params& p, int64_t u, int64_t stages_total, int& tile,
+                                            int64_t& ks0, int64_t& ks1) {
+  int64_t b = u, part = 0, k = 1;
+  if (u >= p.full_units) {
+    k = p.split_k;
+    b = p.full_units + (u - p.full_units) / k;
+    part = (u - p.full_units) % k;
+  }
+  tile = static_cast<int>(b % p.n_tiles);
+  const int64_t c0 = (b / p.n_tiles) * p.kc_stages;
+  const int64_t len = ::min(stages_total, c0 + p.kc_stages) - c0;
+  ks0 = c0 + len * part / k;
+  ks1 = c0 + len * (part + 1) / k;
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
 atb16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
              const __grid_constant__ CUtensorMap mapC, const Params p) {
@@ -282,11 +303,10 @@ atb16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ C
     uint64_t issued = 0;
     bool ok = true;
     for (int64_t u = cid; u < p.units && ok; u += ncl) {
-      const int kc = static_cast<int>(u / p.n_tiles);
-      int ti, tj;
-      decode_tile(p, static_cast<int>(u % p.n_tiles), ti, tj);
-      const int64_t ks0 = static_cast<int64_t>(kc) * p.kc_stages;
-      const int64_t ks1 = ::min((int64_t)stages_total, ks0 + p.kc_stages);
+      int tile, ti, tj;
+      int64_t ks0, ks1;
+      decode_unit(p, u, stages_total, tile, ks0, ks1);
+      decode_tile(p, tile, ti, tj);
       for (int64_t ks = ks0; ks < ks1; ++ks) {
         const int s = static_cast<int>(issued % STAGES);
         const uint32_t ph = static_cast<uint32_t>((issued / STAGES) & 1);
@@ -338,9 +358,9 @@ atb16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ C
       int it = 0;
       bool ok = true;
       for (int64_t u = cid; u < p.units && ok; u += ncl, ++it) {
-        const int kc = static_cast<int>(u / p.n_tiles);
-        const int64_t ks0 = static_cast<int64_t>(kc) * p.kc_stages;
-        const int64_t ks1 = ::min((int64_t)stages_total, ks0 + p.kc_stages);
+        int tile;
+        int64_t ks0, ks1;
+        decode_unit(p, u, stages_total, tile, ks0, ks1);
         const int acc = it & 1;
         int w = 1;
         if (lane == 0) w = mbar_wait_or_abort(&tempty[acc], static_cast<uint32_t>(((it >> 1) & 1) ^ 1), abort_flag);
@@ -399,8 +419,10 @@ atb16_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ C
     int nbuf = 0;
     bool ok = true;
     for (int64_t u = cid; u < p.units; u += ncl, ++it) {
-      int ti, tj;
-      decode_tile(p, static_cast<int>(u % p.n_tiles), ti, tj);
+      int tile, ti, tj;
+      int64_t ks0, ks1;
+      decode_unit(p, u, stages_total, tile, ks0, ks1);
+      decode_tile(p, tile, ti, tj);
       const int acc = it & 1;
       int w = 1;
       if (lane == 0) w = mbar_wait_or_abort(&tfull[acc], static_cast<uint32_t>((it >> 1) & 1), abort_flag) && !*abort_flag;
@@ -625,15 +647,39 @@ void launch_atb16_ex(const Ctx& c, const void* A, const void* B, int64_t n_tok, 
   const int64_t clusters_avail = std::max(1, std::min(ctas / 2, max_clusters[dv]));
 
   const int64_t stages_total = (n_tok + BK - 1) / BK;
-  // Token chunk per unit: long enough to amortise the epilogue, and enough
-  // units (about four per cluster) to balance the clusters.
-  const int64_t want_chunks = std::max<int64_t>(1, (4 * clusters_avail + p.n_tiles - 1) / p.n_tiles);
+  // Token chunk per unit: long enough to amortise the epilogue (at most 8192
+  // tokens, so that the clusters of a round share an L2-sized token window),
+  // and at least one unit per cluster.
+  const int64_t want_chunks = std::max<int64_t>(1, (clusters_avail + p.n_tiles - 1) / p.n_tiles);
   int64_t kcs = (stages_total + want_chunks - 1) / want_chunks;
   kcs = std::max<int64_t>(1024 / BK, std::min<int64_t>(8192 / BK, kcs));
   kcs = std::min(kcs, stages_total);
   p.kc_stages = static_cast<int>(kcs);
   p.n_kc = static_cast<int>((stages_total + kcs - 1) / kcs);
-  p.units = static_cast<int64_t>(p.n_kc) * p.n_tiles;
+  const int64_t chunks = static_cast<int64_t>(p.n_kc) * p.n_tiles;
+  // The units go round the clusters in order.  When the chunks do not fill
+  // the last round, the leftover ones are cut into k parts: a cluster then
+  // ends with ceil(left k / clusters) parts of 1/k chunk instead of one whole
+  // chunk or none (the 256 tiles of a 4096-feature cross product over 70
+  // clusters: 3 chunks + 2 thirds each, in place of 3 or 4 chunks).  Parts
+  // keep at least 8 stages.
+  const int64_t left = chunks % clusters_avail;
+  const int64_t last_len = stages_total - static_cast<int64_t>(p.n_kc - 1) * kcs;
+  const int64_t min_len = left <= p.n_tiles ? last_len : std::min(kcs, last_len);
+  int best_k = 1;
+  if (left > 0) {
+    double best = 1.0;
+    for (int k = 2; k <= 8 && min_len / k >= 8; ++k) {
+      const double load = static_cast<double>((left * k + clusters_avail - 1) / clusters_avail) / k;
+      if (load < best - 1e-9) {
+        best = load;
+        best_k = k;
+      }
+    }
+  }
+  p.split_k = best_k;
+  p.full_units = chunks - (best_k > 1 ? left : 0);
+  p.units = p.full_units + (chunks - p.full_units) * best_k;
   p.alpha = alpha;
   p.status = c.status;
   p.mode = mode;

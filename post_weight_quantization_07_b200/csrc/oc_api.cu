@@ -226,8 +226,13 @@ void gptq_sweep_and_pack(const Ctx& c, float* Wp, int64_t m, int64_t n, const fl
                          float* zeros, unsigned char* codes8, float* Errh, float* Errl, uint32_t* codes,
                          int32_t* perm_out) {
   constexpr int64_t SBW = kSuperBlock;
-  for (int64_t s1 = 0; s1 < n; s1 += SBW) {
-    const int64_t s2 = std::min(n, s1 + SBW);
+  for (int64_t s1 = 0, s2 = 0; s1 < n; s1 = s2) {
+    s2 = std::min(n, s1 + SBW);
+    // A grid taken at a group's first column reads every column of the group,
+    // and only the columns up to the superblock's end have seen all earlier
+    // blocks' errors.  A group wider than a block that does not tile the
+    // superblock (384, 640, 768 ...) therefore starts a superblock of its own.
+    if (!act_order && G > 128 && SBW % G != 0) s2 = std::min(s2, (s1 / G + 1) * G);
     for (int64_t j1 = s1; j1 < s2; j1 += 128) {
       const int64_t bw = std::min<int64_t>(128, s2 - j1);
       const int64_t j2 = j1 + bw;
@@ -417,13 +422,24 @@ int quantize_group(int count, const float* const* W, const int64_t* m, int64_t n
     // QEP makes no dead-column fix: a dead column's correction is zero (its
     // column of d is), so W' keeps W there; GPTQ zeroes it below.
     PhaseScope ps(c, kPhQepApply);
-    launch_permute_w(c, Gl(l), m[l], n, perm, nullptr, Wp);          // G P
-    split_tf32(c, Wp, m[l], n, n, Ph, Pl, n);
+    if (act_order) {
+      launch_permute_w(c, Gl(l), m[l], n, perm, nullptr, Wp);        // G P
+      split_tf32(c, Wp, m[l], n, n, Ph, Pl, n);
+    } else {
+      split_tf32(c, Gl(l), m[l], n, n, Ph, Pl, n);                   // P = I
+    }
     gemm_tf32x3(c, m[l], n, n, 1.f, Ph, Pl, n, Xi, scratch, n, false, Gl(l), n, kBLower);  // T = (G P) Uq^T
     split_tf32(c, Gl(l), m[l], n, n, Ph, Pl, n);
-    launch_permute_w(c, W[l], m[l], n, perm, nullptr, Wp);           // W P
-    gemm_tf32x3(c, m[l], n, n, 2.f * alpha, Ph, Pl, n, UTl, Fs, n, true, Wp, n, kBUpper);
-    launch_permute_w(c, Wp, m[l], n, perm + n, nullptr, W_out[l]);   // back to original order
+    if (act_order) {
+      launch_permute_w(c, W[l], m[l], n, perm, nullptr, Wp);         // W P
+      gemm_tf32x3(c, m[l], n, n, 2.f * alpha, Ph, Pl, n, UTl, Fs, n, true, Wp, n, kBUpper);
+      launch_permute_w(c, Wp, m[l], n, perm + n, nullptr, W_out[l]); // back to original order
+    } else {
+      check_cuda(cudaMemcpyAsync(W_out[l], W[l], static_cast<size_t>(m[l]) * n * sizeof(float),
+                                 cudaMemcpyDeviceToDevice, c.stream),
+                 "copy W");
+      gemm_tf32x3(c, m[l], n, n, 2.f * alpha, Ph, Pl, n, UTl, Fs, n, true, W_out[l], n, kBUpper);
+    }
   }
   {
     // GPTQ with its own factor U (in UTh): U^T split for the trailing updates

@@ -221,12 +221,22 @@ def level_identity(codes_a, zeros_a, codes_b, zeros_b, G):
     return float(np.mean((codes_a - za)[same] == (codes_b - zb)[same]))
 
 
+def oracle_block(n, G):
+    """The oracle's lazy-batch width: 256, or GPTQ's 128 where a group wider
+    than 128 does not tile 256 (a dynamic group must start at a block start or
+    lie inside one block)."""
+    Gn = n if G == -1 else G
+    return 256 if (256 % Gn == 0 or Gn % 256 == 0 or Gn == n) else 128
+
+
 def check_gptq(W, H, wbits, G, damp, act_order, gpu=None):
     codes, scales, zeros, perm, words = gpu if gpu is not None else gpu_gptq(W, H, wbits, G, damp, act_order)
-    ref = oracle.gptq_quantize(W, H, wbits, G, damp, act_order)
+    blk = oracle_block(W.shape[1], G)
+    ref = oracle.gptq_quantize(W, H, wbits, G, damp, act_order, block=blk)
     assert np.array_equal(perm, ref["perm"])
     ident = level_identity(codes, zeros, ref["codes"], ref["zeros"], G)
-    st = oracle.teacher_forced_check(W, H, wbits, G, damp, act_order, codes, scales, zeros, perm=perm)
+    st = oracle.teacher_forced_check(W, H, wbits, G, damp, act_order, codes, scales, zeros, perm=perm,
+                                     block=blk)
     assert st["n_bad"] == 0, st
     assert st["scale_max_rel"] <= SCALE_TOL, st
     assert st["zero_bad"] == 0, st
@@ -243,6 +253,8 @@ def check_gptq(W, H, wbits, G, damp, act_order, gpu=None):
     (64, 256, 3, -1, True),
     (33, 192, 4, -1, False),     # one group of 192 columns across two blocks
     (7, 128, 2, 4, False),       # tiny groups, fewer rows than a CTA's warps
+    (40, 1536, 4, 384, False),   # groups that start inside a 512-column superblock
+    (24, 1536, 3, 768, False),   # and ones that cross into the next superblock
 ])
 def test_gptq_matches_oracle(m, n, wbits, G, act):
     L = random_layer_host(m, n, max(2 * n, 512), seed=1000 + m + n)

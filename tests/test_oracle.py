@@ -279,6 +279,25 @@ def test_gptq_blocked_equals_unblocked(act_order, G):
     assert np.abs(a["deq"] - b["deq"]).max() <= 1e-12 * np.abs(b["deq"]).max()
 
 
+def test_gptq_group_not_tiling_the_block():
+    # a 384-wide group starts inside a 256-column block: the blocked forms take
+    # 128-column blocks, agree with the unblocked definition, and refuse 256
+    L = random_layer_host(24, 768, 1536, seed=19)
+    H = oracle.hessian(L["Xhat"])
+    a = oracle.gptq_quantize(L["W"], H, 4, 384, 0.01, False, block=128)
+    b = oracle.gptq_quantize(L["W"], H, 4, 384, 0.01, False, unblocked=True)
+    assert np.array_equal(a["codes"], b["codes"])
+    assert np.abs(a["scales"] - b["scales"]).max() <= 1e-12 * np.abs(b["scales"]).max()
+    st = oracle.teacher_forced_check(L["W"], H, 4, 384, 0.01, False, a["codes"], a["scales"], a["zeros"],
+                                     block=128)
+    assert st["n_mismatch"] == 0 and st["n_bad"] == 0 and st["scale_max_rel"] <= 1e-12
+    with pytest.raises(ValueError):
+        oracle.gptq_quantize(L["W"], H, 4, 384, 0.01, False, block=256)
+    with pytest.raises(ValueError):
+        oracle.teacher_forced_check(L["W"], H, 4, 384, 0.01, False, a["codes"], a["scales"], a["zeros"],
+                                    block=256)
+
+
 def test_gptq_hessian_scale_invariance():
     L = random_layer_host(16, 256, 512, seed=10)
     H = oracle.hessian(L["Xhat"])
