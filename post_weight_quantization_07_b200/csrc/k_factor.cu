@@ -234,18 +234,24 @@ __global__ void __launch_bounds__(LEAF_THREADS) leaf_chol_inv_kernel(const float
         }
       } else {
         // column c = j - K of Z; rows K + c .. K + 3 of S take its lower part
+        // after the barrier below (every thread is still reading the pivot
+        // block here)
         const int c = j - K;
         w = (c == 0) ? make_float4(z00, z10, z20, z30)
           : (c == 1) ? make_float4(0.f, z11, z21, z31)
           : (c == 2) ? make_float4(0.f, 0.f, z22, z32) : make_float4(0.f, 0.f, 0.f, z33);
-        const float wc[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int r = 0; r < PB; ++r)
-          if (r >= c) S[(K + r) * LDS + j] = wc[r];
       }
       V[j] = w;
     }
     __syncthreads();
+    if (t >= K && t < K + PB) {
+      // the pivot rows are not read again in this step
+      const float4 w = V[t];
+      const float wc[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int r = 0; r < PB; ++r)
+        if (r >= t - K) S[(K + r) * LDS + t] = wc[r];
+    }
     {
       // lane keeps columns j = lane + 32 q and their 4-vectors for the step
       float4 vj[LEAF / 32];

@@ -699,3 +699,25 @@ def test_dequant_gemv_rejects_bad_arguments():
         oc.oc_dequant_gemv(dev(packed.view(np.int32), torch.int32), dev(scales), dev(zeros), 96, 4, 32,
                            dev(x, torch.bfloat16))
     assert e.value.status == oc.OC_ERR_INVALID_ARG
+
+
+def test_factor_and_sweep_repeat_bit_for_bit():
+    """Many factorisation leaves, run again and again: every call succeeds and
+    gives the same codes, scales and zeros bit for bit (the inverse factor and
+    the sweep add nothing through atomics, so any difference would be a race).
+    An 11008-wide H has 86 leaves a call; twelve calls run over a thousand."""
+    n, m = 11008, 64
+    g = torch.Generator(device="cuda").manual_seed(31)
+    Xh = torch.randn(2 * n, n, device="cuda", generator=g)
+    H = 2.0 * (Xh.T @ Xh)
+    W = torch.randn(m, n, device="cuda", generator=g)
+    ref = None
+    for _ in range(12):
+        codes, scales, zeros, _ = oc.oc_gptq_quantize(W, H, 4, 128, 0.01, False)
+        torch.cuda.synchronize()
+        got = (codes.cpu().numpy(), scales.cpu().numpy(), zeros.cpu().numpy())
+        if ref is None:
+            ref = got
+        else:
+            for a, b in zip(ref, got):
+                assert np.array_equal(a, b)
