@@ -105,6 +105,18 @@ int64_t oc_launch_count(void);
  * device stays usable for the next call.  One-shot. */
 int oc_test_inject_stall(void);
 
+/* Test of host logic (no counterpart in the method; touches no device).  How
+ * the tensor-core product over calibration tokens behind the Hessian and the
+ * QEP cross product cuts its work for n_tok tokens, n_tiles output tiles and
+ * `clusters` persistent CTA pairs: units of (tile, token chunk), chunks of
+ * out[0] stages of 128 tokens, out[1] chunks; the units go round the clusters
+ * in order, units [0, out[3]) are whole chunks and each later one is one of
+ * out[2] equal parts of a leftover chunk, out[4] units in all.
+ *   out  int64 [5], host memory, written.
+ * Returns OC_ERR_INVALID_ARG unless n_tok, n_tiles and clusters are positive
+ * and out is non-null. */
+int oc_test_unit_plan(int64_t n_tok, int64_t n_tiles, int64_t clusters, int64_t* out);
+
 /*
  * Hessian accumulation:  H += 2 * X^T X   (n x n, fp32)
  *

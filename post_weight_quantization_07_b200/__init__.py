@@ -20,7 +20,8 @@ __all__ = ["OC_OK", "OC_ERR_INVALID_ARG", "OC_ERR_UNSUPPORTED", "OC_ERR_NOT_SPD"
            "oc_qep_correct", "oc_gptq_quantize", "oc_set_sync", "oc_stream_status",
            "oc_workspace_release", "oc_status_string", "oc_last_error", "oc_version",
            "oc_profile_enable", "oc_profile_read", "oc_launch_count", "oc_quantize_layer",
-           "oc_lpcd_left_project", "lpcd_pair", "oc_dequant_gemv", "oc_test_inject_stall"]
+           "oc_lpcd_left_project", "lpcd_pair", "oc_dequant_gemv", "oc_test_inject_stall",
+           "oc_test_unit_plan"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liboc.so")
@@ -73,6 +74,8 @@ def _load():
     L.oc_launch_count.restype = i64
     L.oc_test_inject_stall.argtypes = []
     L.oc_test_inject_stall.restype = i32
+    L.oc_test_unit_plan.argtypes = [i64, i64, i64, vp]
+    L.oc_test_unit_plan.restype = i32
     L.oc_hessian_accumulate.argtypes = [vp, i64, i64, vp, vp]
     L.oc_hessian_accumulate.restype = i32
     L.oc_qep_correct.argtypes = [vp, i64, i64, vp, vp, i64, f32, f32, vp, vp, vp]
@@ -183,6 +186,15 @@ def oc_test_inject_stall() -> None:
     """Make the next tensor-core product launch stall on a barrier nothing
     releases: its bounded wait runs out and the call reports OC_ERR_TIMEOUT."""
     _check(_lib().oc_test_inject_stall(), "oc_test_inject_stall")
+
+
+def oc_test_unit_plan(n_tok, n_tiles, clusters):
+    """How the tensor-core product over tokens cuts its work (host logic only):
+    returns (kc_stages, n_kc, split_k, full_units, units)."""
+    out = (ctypes.c_int64 * 5)()
+    _check(_lib().oc_test_unit_plan(int(n_tok), int(n_tiles), int(clusters), ctypes.cast(out, ctypes.c_void_p)),
+           "oc_test_unit_plan")
+    return tuple(int(v) for v in out)
 
 
 def oc_workspace_release() -> None:

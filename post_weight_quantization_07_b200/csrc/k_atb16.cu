@@ -646,40 +646,12 @@ void launch_atb16_ex(const Ctx& c, const void* A, const void* B, int64_t n_tok, 
   const int ctas = (max_ctas > 0 && max_ctas < c.sm_count) ? max_ctas : c.sm_count;
   const int64_t clusters_avail = std::max(1, std::min(ctas / 2, max_clusters[dv]));
 
-  const int64_t stages_total = (n_tok + BK - 1) / BK;
-  // Token chunk per unit: long enough to amortise the epilogue (at most 8192
-  // tokens, so that the clusters of a round share an L2-sized token window),
-  // and at least one unit per cluster.
-  const int64_t want_chunks = std::max<int64_t>(1, (clusters_avail + p.n_tiles - 1) / p.n_tiles);
-  int64_t kcs = (stages_total + want_chunks - 1) / want_chunks;
-  kcs = std::max<int64_t>(1024 / BK, std::min<int64_t>(8192 / BK, kcs));
-  kcs = std::min(kcs, stages_total);
-  p.kc_stages = static_cast<int>(kcs);
-  p.n_kc = static_cast<int>((stages_total + kcs - 1) / kcs);
-  const int64_t chunks = static_cast<int64_t>(p.n_kc) * p.n_tiles;
-  // The units go round the clusters in order.  When the chunks do not fill
-  // the last round, the leftover ones are cut into k parts: a cluster then
-  // ends with ceil(left k / clusters) parts of 1/k chunk instead of one whole
-  // chunk or none (the 256 tiles of a 4096-feature cross product over 70
-  // clusters: 3 chunks + 2 thirds each, in place of 3 or 4 chunks).  Parts
-  // keep at least 8 stages.
-  const int64_t left = chunks % clusters_avail;
-  const int64_t last_len = stages_total - static_cast<int64_t>(p.n_kc - 1) * kcs;
-  const int64_t min_len = left <= p.n_tiles ? last_len : std::min(kcs, last_len);
-  int best_k = 1;
-  if (left > 0) {
-    double best = 1.0;
-    for (int k = 2; k <= 8 && min_len / k >= 8; ++k) {
-      const double load = static_cast<double>((left * k + clusters_avail - 1) / clusters_avail) / k;
-      if (load < best - 1e-9) {
-        best = load;
-        best_k = k;
-      }
-    }
-  }
-  p.split_k = best_k;
-  p.full_units = chunks - (best_k > 1 ? left : 0);
-  p.units = p.full_units + (chunks - p.full_units) * best_k;
+  const UnitPlan plan = plan_units(n_tok, p.n_tiles, clusters_avail);
+  p.kc_stages = static_cast<int>(plan.kc_stages);
+  p.n_kc = static_cast<int>(plan.n_kc);
+  p.split_k = plan.split_k;
+  p.full_units = plan.full_units;
+  p.units = plan.units;
   p.alpha = alpha;
   p.status = c.status;
   p.mode = mode;
@@ -710,6 +682,45 @@ void launch_atb16_ex(const Ctx& c, const void* A, const void* B, int64_t n_tok, 
 }
 
 }  // namespace
+
+UnitPlan plan_units(int64_t n_tok, int64_t n_tiles, int64_t clusters) {
+  UnitPlan u{};
+  const int64_t stages_total = (n_tok + BK - 1) / BK;
+  // Token chunk per unit: long enough to amortise the epilogue (at most 8192
+  // tokens, so that the clusters of a round share an L2-sized token window),
+  // and at least one unit per cluster.
+  const int64_t want_chunks = std::max<int64_t>(1, (clusters + n_tiles - 1) / n_tiles);
+  int64_t kcs = (stages_total + want_chunks - 1) / want_chunks;
+  kcs = std::max<int64_t>(1024 / BK, std::min<int64_t>(8192 / BK, kcs));
+  kcs = std::min(kcs, stages_total);
+  u.kc_stages = kcs;
+  u.n_kc = (stages_total + kcs - 1) / kcs;
+  const int64_t chunks = u.n_kc * n_tiles;
+  // The units go round the clusters in order.  When the chunks do not fill
+  // the last round, the leftover ones are cut into k parts: a cluster then
+  // ends with ceil(left k / clusters) parts of 1/k chunk instead of one whole
+  // chunk or none (the 256 tiles of a 4096-feature cross product over 70
+  // clusters: 3 chunks + 2 thirds each, in place of 3 or 4 chunks).  Parts
+  // keep at least 8 stages.
+  const int64_t left = chunks % clusters;
+  const int64_t last_len = stages_total - (u.n_kc - 1) * kcs;
+  const int64_t min_len = left <= n_tiles ? last_len : std::min(kcs, last_len);
+  int best_k = 1;
+  if (left > 0) {
+    double best = 1.0;
+    for (int k = 2; k <= 8 && min_len / k >= 8; ++k) {
+      const double load = static_cast<double>((left * k + clusters - 1) / clusters) / k;
+      if (load < best - 1e-9) {
+        best = load;
+        best_k = k;
+      }
+    }
+  }
+  u.split_k = best_k;
+  u.full_units = chunks - (best_k > 1 ? left : 0);
+  u.units = u.full_units + (chunks - u.full_units) * best_k;
+  return u;
+}
 
 void request_test_stall() { g_stall_request = true; }
 

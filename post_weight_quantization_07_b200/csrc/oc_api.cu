@@ -522,6 +522,20 @@ int oc_test_inject_stall(void) {
   });
 }
 
+int oc_test_unit_plan(int64_t n_tok, int64_t n_tiles, int64_t clusters, int64_t* out) {
+  return guarded([&]() -> int {
+    if (n_tok <= 0 || n_tiles <= 0 || clusters <= 0 || out == nullptr)
+      fail(OC_ERR_INVALID_ARG, "unit plan: n_tok, n_tiles and clusters must be positive, out non-null");
+    const UnitPlan u = plan_units(n_tok, n_tiles, clusters);
+    out[0] = u.kc_stages;
+    out[1] = u.n_kc;
+    out[2] = u.split_k;
+    out[3] = u.full_units;
+    out[4] = u.units;
+    return OC_OK;
+  });
+}
+
 int oc_workspace_release(void) {
   return guarded([&]() -> int {
     int dev = 0;

@@ -109,6 +109,16 @@ CUtensorMap make_tmap_2d(const void* base, CUtensorMapDataType dt, int elem_byte
 void launch_atb16(const Ctx& c, const void* A, const void* B, int64_t n_tok, int64_t M, int64_t N, float alpha,
                   float* C, int64_t ldc, bool upper_only, int max_ctas = 0);
 
+// How a persistent tensor-core product over tokens cuts its work: units of
+// (output tile, token chunk of kc_stages 128-token stages, n_kc chunks),
+// taken round-robin by `clusters` CTA pairs; units [0, full_units) are whole
+// chunks, the rest split_k parts of the leftover chunks (units in all).
+struct UnitPlan {
+  int64_t kc_stages, n_kc, full_units, units;
+  int split_k;
+};
+UnitPlan plan_units(int64_t n_tok, int64_t n_tiles, int64_t clusters);
+
 // The next launch_atb16 / launch_cross_product launch of the tensor-core
 // product stalls on a barrier nothing releases (test of the failure path).
 void request_test_stall();
