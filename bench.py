@@ -451,9 +451,11 @@ def run_ours(args, rank, world, local_rank):
         step_three_calls()
     g1.record(stream)
     barrier()
+    # A failure in this or the later side measurements is reported in the line
+    # (with no figure for that measurement); only the timed steps' own failure
+    # stops the run.  Every rank still takes the same collective steps.
     st = oc.oc_stream_status(stream)
-    if st != oc.OC_OK:
-        raise RuntimeError(f"three-call steps failed: {oc.oc_status_string(st)}")
+    three_err = None if st == oc.OC_OK else f"three-call steps failed: {oc.oc_status_string(st)}"
     ms_three = max_over_ranks(g0.elapsed_time(g1)) / args.steps
 
     # ---- end to end: pinned host inputs copied in and results read back every step
@@ -488,13 +490,14 @@ def run_ours(args, rank, world, local_rank):
         f1.record(stream)
         barrier()
         st = oc.oc_stream_status(stream)
-        if st != oc.OC_OK:
-            raise RuntimeError(f"end-to-end steps failed: {oc.oc_status_string(st)}")
         ms_e2e = max_over_ranks(f0.elapsed_time(f1))
         h2d = Xh.numel() * Xh.element_size() + X.numel() * X.element_size() + W.numel() * 4
         d2h = codes.numel() * 4 + scales.numel() * 4 + zeros.numel() * 4
         e2e = {"value": world * k2 / (ms_e2e / 1e3), "unit": UNIT, "steps": k2,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+        if st != oc.OC_OK:
+            e2e["value"] = None
+            e2e["error"] = f"end-to-end steps failed: {oc.oc_status_string(st)}"
 
     # ---- the 224 layers of a 7B-shaped model, each on its own inputs
     model = None
@@ -592,13 +595,15 @@ def run_ours(args, rank, world, local_rank):
         "config": dict(workload_config(spec),
                        parallelism=(f"{world} independent layers, one per rank" if world > 1
                                     else "single GPU")),
-        "seconds_per_7b_model": model["seconds"] if model else None,
+        "seconds_per_7b_model": model.get("seconds") if model else None,
         "model_pass": model,
         "seconds_per_224_layers_of_this_shape": round(224 * ms_per_step / 1e3, 3),
-        "three_calls_ms_per_step": round(ms_three, 3),
+        "three_calls_ms_per_step": round(ms_three, 3) if three_err is None else None,
         "roofline": roof, "layer_roofline": layer_roof, "phases": phase_out, "gpu_launches": int(launches),
         "clocks": clocks, "e2e": e2e,
     }
+    if three_err is not None:
+        line["three_calls_error"] = three_err
     if args.rotate:
         line["config"]["rotation"] = (f"block-{args.rotate} Hadamard rotation of W, X and Xhat in every step "
                                       f"(oc_hadamard_rotate), the layer quantised in the rotated basis")
@@ -649,10 +654,10 @@ def model_pass(args, rank, world, stream, barrier, max_over_ranks):
         done += 1
         del L, outs
     st = oc.oc_stream_status(stream)
-    if st != oc.OC_OK:
-        raise RuntimeError(f"model pass failed: {oc.oc_status_string(st)}")
     barrier()
     ms = max_over_ranks(total_ms)
+    if st != oc.OC_OK:
+        return {"seconds": None, "error": f"model pass failed: {oc.oc_status_string(st)}", "layers": len(specs)}
     return {"seconds": round(ms / 1e3, 3), "layers": len(specs), "layers_per_rank": done,
             "layers_per_s": round(len(specs) / (ms / 1e3), 3), "calibration_tokens": args.model_tokens,
             "gpu_launches": int(oc.oc_launch_count() - launches0),
