@@ -38,7 +38,9 @@
 //                it with plain 16-byte loads and stores (no shared memory,
 //                which the ring fills).
 // Work units are (output tile, token chunk); chunks are the outer index so
-// that the clusters of one wave stream the same token window through L2.
+// that the clusters of one wave stream the same token window through L2, and
+// the chunks of a last, partly filled round are cut into equal parts so that
+// it spreads over every cluster (plan_units).
 // Every wait is bounded; a wait that gives up records OC_ERR_TIMEOUT and the
 // kernel winds down (both CTAs still meet at the final cluster barrier).
 //
